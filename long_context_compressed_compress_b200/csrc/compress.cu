@@ -1,0 +1,401 @@
+// Streaming kernels of the CSA/HCA layer: the gated overlapping 4:1 compressor
+// (cf-1.com/news/5231315 §3.1), the 128:1 compressor (§3.2), NVFP4 block
+// quantisation of the indexer QK path (§3.4, §4.4), and the decode-state
+// helpers (ring append, position advance; §4.4 KV cache tiers).
+//
+// All of these are HBM-bound: one thread owns 8 channels of one entry and
+// moves 16-byte vectors, consecutive threads cover consecutive channels so a
+// warp reads whole contiguous rows.
+#include "common.cuh"
+
+namespace csa {
+
+__device__ int g_dev_status = 0;
+
+static thread_local int t_last_cuda_error = 0;
+
+int* device_status_ptr() {
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+int set_cuda_error(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return CSA_ERR_CUDA;
+}
+int check_launch() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? CSA_OK : set_cuda_error(e);
+}
+
+// ---------------------------------------------------------------------------
+// csa_compress: thread = (b, entry, 8-channel group).  Two passes over the 2m
+// rows of the block pair: the per-channel max of the gate logits, then the
+// exp-weighted sums of a (current block) and b (predecessor block).
+// ---------------------------------------------------------------------------
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) csa_compress_kernel(
+    const Tin* __restrict__ a, const Tin* __restrict__ b, const Tin* __restrict__ z, int B, int T, int D, int m,
+    int fhp, int S, const int32_t* __restrict__ ring_pos, int out_bstride, Tout* __restrict__ out,
+    uint8_t* __restrict__ out_fp4, uint8_t* __restrict__ out_sf, float g) {
+  const int G = D >> 3;
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const bool decode = ring_pos != nullptr;
+  const long long total = decode ? static_cast<long long>(B) * G : static_cast<long long>(B) * S * G;
+  const bool valid = gid < total;
+  const long long g2 = valid ? gid : 0;
+  const int cg = static_cast<int>(g2 % G);
+  long long eidx;   // entry index written (within the batch row)
+  int bi;
+  // row offsets (within the batch's [rows, D] slab) of the current / predecessor blocks
+  int cur0, pred0, has_pred;
+  bool active = valid;
+  if (!decode) {
+    const long long e = (g2 / G) % S;
+    bi = static_cast<int>(g2 / (static_cast<long long>(G) * S));
+    const int blk = static_cast<int>(e) + fhp;
+    cur0 = m * blk;
+    pred0 = m * (blk - 1);
+    has_pred = blk > 0;
+    eidx = e;
+  } else {
+    bi = static_cast<int>(g2 / G);
+    const int p = ring_pos[bi];
+    active = valid && ((p + 1) % m == 0);
+    const int i = (p + 1) / m - 1;
+    cur0 = (i & 1) * m;
+    pred0 = ((i + 1) & 1) * m;
+    has_pred = i > 0;
+    eidx = i;
+  }
+  const int rows = decode ? 2 * m : T;
+  const size_t slab = static_cast<size_t>(bi) * rows * D + static_cast<size_t>(cg) * 8;
+  const Tin* zb = z + slab;
+  float mx[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
+  float v[8];
+  if (active) {
+    for (int r = 0; r < m; ++r) {
+      Vec8<Tin>::load(zb + static_cast<size_t>(cur0 + r) * D, v);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], v[c]);
+      if (has_pred) {
+        Vec8<Tin>::load(zb + static_cast<size_t>(pred0 + r) * D, v);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], v[c]);
+      }
+    }
+  }
+  float sum[8], acc[8], x[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) { sum[c] = 0.f; acc[c] = 0.f; }
+  if (active) {
+    for (int r = 0; r < m; ++r) {
+      Vec8<Tin>::load(zb + static_cast<size_t>(cur0 + r) * D, v);
+      Vec8<Tin>::load(a + slab + static_cast<size_t>(cur0 + r) * D, x);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float e = expf(v[c] - mx[c]);
+        sum[c] += e;
+        acc[c] = fmaf(e, x[c], acc[c]);
+      }
+      if (has_pred) {
+        Vec8<Tin>::load(zb + static_cast<size_t>(pred0 + r) * D, v);
+        Vec8<Tin>::load(b + slab + static_cast<size_t>(pred0 + r) * D, x);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float e = expf(v[c] - mx[c]);
+          sum[c] += e;
+          acc[c] = fmaf(e, x[c], acc[c]);
+        }
+      }
+    }
+  }
+  float e8[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) e8[c] = active ? round_to(__fdiv_rn(acc[c], sum[c]), (Tout*)nullptr) : 0.f;
+  const size_t orow = static_cast<size_t>(bi) * out_bstride + static_cast<size_t>(eidx);
+  if (out != nullptr && active) Vec8<Tout>::store(out + orow * D + cg * 8, e8);
+  if (out_fp4 != nullptr) {
+    // 16-element NVFP4 block = this thread's 8 channels + its neighbour's.
+    float am = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) am = fmaxf(am, fabsf(e8[c]));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    uint32_t sfb;
+    const uint32_t codes = nvfp4_encode8(e8, am, g, &sfb);
+    if (active) {
+      reinterpret_cast<uint32_t*>(out_fp4 + orow * (D / 2))[cg] = codes;
+      if ((cg & 1) == 0) out_sf[orow * (D / 16) + (cg >> 1)] = static_cast<uint8_t>(sfb);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// hca_compress: CTA = (b, entry).  Thread (rg, cg) reduces rows rg, rg+RG, ...
+// of the block for 8 channels (max, then exp-sums with its own max); the RG
+// partial (max, sum, acc) triples are merged in shared memory.
+// ---------------------------------------------------------------------------
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) hca_compress_kernel(const Tin* __restrict__ a, const Tin* __restrict__ z,
+                                                           int T, int D, int m, int S, Tout* __restrict__ out) {
+  extern __shared__ float sm[];
+  const int G = D >> 3;
+  const int RG = blockDim.x / G;
+  const int cg = threadIdx.x % G;
+  const int rg = threadIdx.x / G;
+  const int e = blockIdx.x % S;
+  const int bi = blockIdx.x / S;
+  const size_t base = (static_cast<size_t>(bi) * T + static_cast<size_t>(e) * m) * D + cg * 8;
+  float mx[8], sum[8], acc[8], v[8], x[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) { mx[c] = -INFINITY; sum[c] = 0.f; acc[c] = 0.f; }
+  for (int r = rg; r < m; r += RG) {
+    Vec8<Tin>::load(z + base + static_cast<size_t>(r) * D, v);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], v[c]);
+  }
+  for (int r = rg; r < m; r += RG) {
+    Vec8<Tin>::load(z + base + static_cast<size_t>(r) * D, v);
+    Vec8<Tin>::load(a + base + static_cast<size_t>(r) * D, x);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float ex = expf(v[c] - mx[c]);
+      sum[c] += ex;
+      acc[c] = fmaf(ex, x[c], acc[c]);
+    }
+  }
+  // partials: sm[(rg*3 + {0,1,2}) * D + channel]
+  const int ch = cg * 8;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    sm[(rg * 3 + 0) * D + ch + c] = mx[c];
+    sm[(rg * 3 + 1) * D + ch + c] = sum[c];
+    sm[(rg * 3 + 2) * D + ch + c] = acc[c];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    float M = -INFINITY;
+    for (int r = 0; r < RG; ++r) M = fmaxf(M, sm[(r * 3) * D + c]);
+    float Ssum = 0.f, A = 0.f;
+    for (int r = 0; r < RG; ++r) {
+      const float mr = sm[(r * 3) * D + c];
+      if (mr == -INFINITY) continue;     // row group saw no rows (m < RG)
+      const float f = expf(mr - M);
+      Ssum = fmaf(sm[(r * 3 + 1) * D + c], f, Ssum);
+      A = fmaf(sm[(r * 3 + 2) * D + c], f, A);
+    }
+    const float val = __fdiv_rn(A, Ssum);
+    Tout* o = out + (static_cast<size_t>(bi) * S + e) * D + c;
+    *o = static_cast<Tout>(val);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// nvfp4_quantize: thread = 8 elements; pairs of threads share a 16-block.
+// ---------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(256) nvfp4_quantize_kernel(const Tin* __restrict__ x, long long n8, float g,
+                                                             uint8_t* __restrict__ packed,
+                                                             uint8_t* __restrict__ sf) {
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const bool valid = gid < n8;
+  float v[8];
+  if (valid) {
+    Vec8<Tin>::load(x + gid * 8, v);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) v[c] = 0.f;
+  }
+  float am = 0.f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) am = fmaxf(am, fabsf(v[c]));
+  am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+  uint32_t sfb;
+  const uint32_t codes = nvfp4_encode8(v, am, g, &sfb);
+  if (valid) {
+    reinterpret_cast<uint32_t*>(packed)[gid] = codes;
+    if ((gid & 1) == 0) sf[gid >> 1] = static_cast<uint8_t>(sfb);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// decode helpers
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void ring_append_kernel(const T* __restrict__ rows, int B, int D, T* __restrict__ ring, int cap,
+                                   const int32_t* __restrict__ pos) {
+  const int bi = blockIdx.x;
+  const int slot = pos[bi] % cap;
+  for (int c = threadIdx.x; c < D; c += blockDim.x)
+    ring[(static_cast<size_t>(bi) * cap + slot) * D + c] = rows[static_cast<size_t>(bi) * D + c];
+}
+
+__global__ void pos_advance_kernel(int32_t* pos, int B, int delta) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < B) pos[i] += delta;
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+// ============================================================== C ABI entries
+extern "C" {
+
+const char* csa_status_string(int status) {
+  switch (status) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_INVALID_ARG: return "CSA_ERR_INVALID_ARG";
+    case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
+    case CSA_ERR_ALIGNMENT: return "CSA_ERR_ALIGNMENT";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+    case CSA_ERR_TIMEOUT: return "CSA_ERR_TIMEOUT";
+    default: return "CSA_ERR_UNKNOWN";
+  }
+}
+
+int csa_last_cuda_error(void) { return t_last_cuda_error; }
+
+int csa_version(void) { return 100; }
+
+int csa_device_status(int* status_out) {
+  if (status_out == nullptr) return CSA_ERR_INVALID_ARG;
+  int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(int));
+  if (e != cudaSuccess) return set_cuda_error(e);
+  e = cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return set_cuda_error(e);
+  *status_out = v;
+  return CSA_OK;
+}
+
+int csa_compress(const void* a, const void* b, const void* z, int in_dtype, int B, int T, int D, int m,
+                 int first_has_pred, const int32_t* ring_pos, int out_bstride, void* out, int out_dtype,
+                 uint8_t* out_fp4, uint8_t* out_sf, float gscale, csa_stream_t stream) {
+  CSA_REQUIRE(a && b && z, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(out || out_fp4, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(B >= 0 && T >= 0 && D > 0 && m >= 1 && m <= 16, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(in_dtype == CSA_F32 || in_dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(out_dtype == CSA_F32 || out_dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(D % 8 == 0, CSA_ERR_UNSUPPORTED);
+  CSA_REQUIRE(aligned16(a) && aligned16(b) && aligned16(z), CSA_ERR_ALIGNMENT);
+  CSA_REQUIRE(!out || aligned16(out), CSA_ERR_ALIGNMENT);
+  if (out_fp4) {
+    CSA_REQUIRE(out_sf != nullptr && gscale > 0.f, CSA_ERR_INVALID_ARG);
+    CSA_REQUIRE(D % 16 == 0, CSA_ERR_UNSUPPORTED);
+    CSA_REQUIRE((reinterpret_cast<uintptr_t>(out_fp4) & 3u) == 0, CSA_ERR_ALIGNMENT);
+  }
+  const bool decode = ring_pos != nullptr;
+  int S = 0;
+  if (!decode) {
+    CSA_REQUIRE(first_has_pred == 0 || first_has_pred == 1, CSA_ERR_INVALID_ARG);
+    S = T / m - first_has_pred;
+    if (S <= 0 || B == 0) return CSA_OK;
+    if (out_bstride == 0) out_bstride = S;
+    CSA_REQUIRE(out_bstride >= S, CSA_ERR_INVALID_ARG);
+  } else {
+    CSA_REQUIRE(out_bstride > 0, CSA_ERR_INVALID_ARG);
+    if (B == 0) return CSA_OK;
+  }
+  const long long threads = decode ? static_cast<long long>(B) * (D / 8) : static_cast<long long>(B) * S * (D / 8);
+  const int bs = 256;
+  const long long grid = (threads + bs - 1) / bs;
+  CSA_REQUIRE(grid < (1ll << 31), CSA_ERR_UNSUPPORTED);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define CSA_LAUNCH_COMPRESS(TI, TO)                                                                       \
+  csa_compress_kernel<TI, TO><<<static_cast<unsigned>(grid), bs, 0, st>>>(                               \
+      static_cast<const TI*>(a), static_cast<const TI*>(b), static_cast<const TI*>(z), B, T, D, m,       \
+      first_has_pred, S, ring_pos, out_bstride, static_cast<TO*>(out), out_fp4, out_sf, gscale)
+  if (in_dtype == CSA_F32 && out_dtype == CSA_F32) CSA_LAUNCH_COMPRESS(float, float);
+  else if (in_dtype == CSA_F32) CSA_LAUNCH_COMPRESS(float, __nv_bfloat16);
+  else if (out_dtype == CSA_F32) CSA_LAUNCH_COMPRESS(__nv_bfloat16, float);
+  else CSA_LAUNCH_COMPRESS(__nv_bfloat16, __nv_bfloat16);
+#undef CSA_LAUNCH_COMPRESS
+  return check_launch();
+}
+
+int hca_compress(const void* a, const void* z, int in_dtype, int B, int T, int D, int m, void* out,
+                 int out_dtype, csa_stream_t stream) {
+  CSA_REQUIRE(a && z && out, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(B >= 0 && T >= 0 && D > 0 && m >= 1, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(in_dtype == CSA_F32 || in_dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(out_dtype == CSA_F32 || out_dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(D % 8 == 0 && D <= 2048, CSA_ERR_UNSUPPORTED);
+  CSA_REQUIRE(aligned16(a) && aligned16(z), CSA_ERR_ALIGNMENT);
+  const int S = T / m;
+  if (S == 0 || B == 0) return CSA_OK;
+  const long long grid = static_cast<long long>(B) * S;
+  CSA_REQUIRE(grid < (1ll << 31), CSA_ERR_UNSUPPORTED);
+  const int G = D / 8;
+  int RG = 256 / G;
+  if (RG < 1) RG = 1;
+  const int bs = G * RG;
+  const size_t smem = static_cast<size_t>(RG) * 3 * D * sizeof(float);
+  CSA_REQUIRE(smem <= 48 * 1024, CSA_ERR_UNSUPPORTED);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define CSA_LAUNCH_HCA(TI, TO)                                                                        \
+  hca_compress_kernel<TI, TO><<<static_cast<unsigned>(grid), bs, smem, st>>>(                        \
+      static_cast<const TI*>(a), static_cast<const TI*>(z), T, D, m, S, static_cast<TO*>(out))
+  if (in_dtype == CSA_F32 && out_dtype == CSA_F32) CSA_LAUNCH_HCA(float, float);
+  else if (in_dtype == CSA_F32) CSA_LAUNCH_HCA(float, __nv_bfloat16);
+  else if (out_dtype == CSA_F32) CSA_LAUNCH_HCA(__nv_bfloat16, float);
+  else CSA_LAUNCH_HCA(__nv_bfloat16, __nv_bfloat16);
+#undef CSA_LAUNCH_HCA
+  return check_launch();
+}
+
+int nvfp4_quantize(const void* x, int in_dtype, int64_t rows, int D, float gscale, uint8_t* packed,
+                   uint8_t* sf, csa_stream_t stream) {
+  CSA_REQUIRE(x && packed && sf, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(rows >= 0 && D > 0 && gscale > 0.f, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(in_dtype == CSA_F32 || in_dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(D % 16 == 0, CSA_ERR_UNSUPPORTED);
+  CSA_REQUIRE(aligned16(x) && (reinterpret_cast<uintptr_t>(packed) & 3u) == 0, CSA_ERR_ALIGNMENT);
+  const long long n8 = rows * (D / 8);
+  if (n8 == 0) return CSA_OK;
+  const int bs = 256;
+  const long long grid = (n8 + bs - 1) / bs;
+  CSA_REQUIRE(grid < (1ll << 31), CSA_ERR_UNSUPPORTED);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (in_dtype == CSA_F32)
+    nvfp4_quantize_kernel<float><<<static_cast<unsigned>(grid), bs, 0, st>>>(static_cast<const float*>(x), n8,
+                                                                             gscale, packed, sf);
+  else
+    nvfp4_quantize_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), bs, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), n8, gscale, packed, sf);
+  return check_launch();
+}
+
+int csa_ring_append(const void* rows, int dtype, int B, int D, void* ring, int cap, const int32_t* pos,
+                    csa_stream_t stream) {
+  CSA_REQUIRE(rows && ring && pos, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(B >= 0 && D > 0 && cap > 0, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
+  if (B == 0) return CSA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == CSA_F32)
+    ring_append_kernel<float><<<B, 128, 0, st>>>(static_cast<const float*>(rows), B, D, static_cast<float*>(ring),
+                                                 cap, pos);
+  else
+    ring_append_kernel<__nv_bfloat16><<<B, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(rows), B, D,
+                                                         static_cast<__nv_bfloat16*>(ring), cap, pos);
+  return check_launch();
+}
+
+int csa_pos_advance(int32_t* pos, int B, int delta, csa_stream_t stream) {
+  CSA_REQUIRE(pos != nullptr && B >= 0, CSA_ERR_INVALID_ARG);
+  if (B == 0) return CSA_OK;
+  pos_advance_kernel<<<(B + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(pos, B, delta);
+  return check_launch();
+}
+
+}  // extern "C"

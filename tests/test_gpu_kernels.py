@@ -1,0 +1,333 @@
+"""GPU parity of each entry point against the CPU oracle, through the C ABI.
+
+Sizes span several tiles plus ragged tails.  Tolerances:
+  * NVFP4 codes/scales and top-k indices: bit-exact;
+  * fp32 results: 1e-5 * max(1, |ref|) (spec fp32 bound);
+  * bf16 results: the bf16 rounding of the oracle value within one bf16 ulp
+    for single-rounding steps (compressors, scores), 2e-2 max-abs for
+    attention outputs (spec bf16 bound).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import formats
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@pytest.fixture(scope="module")
+def ops(cuda_ok):
+    from long_context_compressed_compress_b200 import build
+    build.build()
+    from long_context_compressed_compress_b200 import ops as o
+    return o
+
+
+def _randn(shape, dtype, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(DT[dtype])
+
+
+def _np(t):
+    return t.detach().cpu().to(torch.float64).numpy()
+
+
+def _ulp_bf16(x):
+    """One bf16 ulp at |x| (power-of-two spacing; 2^-133 floor)."""
+    x = np.maximum(np.abs(x), 2.0 ** -126)
+    _, e = np.frexp(x)
+    return np.ldexp(1.0, e - 1 - 7)
+
+
+def _assert_close(got, ref, dtype):
+    if dtype == "f32":
+        tol = 1e-5 * np.maximum(1.0, np.abs(ref))
+        bad = np.abs(got - ref) > tol
+    else:
+        bad = np.abs(got - ref) > _ulp_bf16(ref) * 1.0 + 1e-30
+    assert not bad.any(), f"{bad.sum()} mismatches; max err {np.abs(got - ref).max():.3e}"
+
+
+# ------------------------------------------------------------------ NVFP4
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_nvfp4_quantize_bit_exact(ops, dtype):
+    rows, D = 1000, 64
+    x = _randn((rows, D), dtype, 1) * torch.exp(_randn((rows, 1), "f32", 2) * 3).to(DT[dtype])
+    x = x.to(DT[dtype])
+    x[0] = 0                                   # all-zero blocks
+    x[1, :16] = torch.tensor([6.0, -4, 3, -2, 1.5, -1, 0.5, 0, 5, -5, 2.5, -2.5, 1.25, 0.75, 0.25, 0.1])
+    x[2, :16] = 1e-30 if dtype == "f32" else 1e-30   # scale underflows in E4M3
+    x[3, :16] = 3e4                            # scale saturates at 448
+    for g in (1.0, 0.37):
+        xd = x.cuda()
+        packed = torch.empty((rows, D // 2), dtype=torch.uint8, device="cuda")
+        sf = torch.empty((rows, D // 16), dtype=torch.uint8, device="cuda")
+        ops.nvfp4_quantize(xd, packed, sf, gscale=g)
+        ref = oracle.nvfp4_quantize(x, g)
+        np.testing.assert_array_equal(sf.cpu().numpy(), ref["sf"])
+        got = packed.cpu().numpy()
+        # +0/-0 codes are the same value; compare canonicalised nibbles and raw bytes
+        lo, hi = got & 0xF, got >> 4
+        canon = lambda c: np.where(c == 8, 0, c)
+        np.testing.assert_array_equal(canon(lo), canon(ref["codes"][:, 0::2]))
+        np.testing.assert_array_equal(canon(hi), canon(ref["codes"][:, 1::2]))
+
+
+def test_e2m1_rounding_every_midpoint_on_gpu(ops):
+    """Every E2M1 midpoint and its fp32 neighbours, with scale 1 (amax = 6)."""
+    g = formats.E2M1_VALUES
+    mids = (g[1:] + g[:-1]) / 2
+    vals = np.concatenate([mids, np.nextafter(mids.astype(np.float32), np.float32(0)),
+                           np.nextafter(mids.astype(np.float32), np.float32(9)), g]).astype(np.float32)
+    vals = np.concatenate([vals, -vals])
+    n = (len(vals) + 14) // 15 * 15
+    pad = np.zeros(n, dtype=np.float32)
+    pad[: len(vals)] = vals
+    blocks = pad.reshape(-1, 15)
+    x = np.concatenate([np.full((blocks.shape[0], 1), 6.0, np.float32), blocks], axis=1)   # amax = 6 -> s = 1
+    xt = torch.from_numpy(x).cuda()
+    packed = torch.empty((x.shape[0], 8), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((x.shape[0], 1), dtype=torch.uint8, device="cuda")
+    ops.nvfp4_quantize(xt, packed, sf, 1.0)
+    ref = oracle.nvfp4_quantize(x, 1.0)
+    got = packed.cpu().numpy()
+    codes = np.stack([got & 0xF, got >> 4], -1).reshape(x.shape)
+    dec = formats.e2m1_decode(codes) * formats.e4m3_decode(sf.cpu().numpy())
+    np.testing.assert_array_equal(dec, ref["xhat"])
+
+
+# ------------------------------------------------------------- compressors
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("B,T,D", [(1, 1030, 64), (2, 517, 128)])
+def test_csa_compress(ops, dtype, B, T, D):
+    m = 4
+    a, b, z = (_randn((B, T, D), dtype, s) for s in (3, 4, 5))
+    S = T // m
+    out = torch.empty((B, S, D), dtype=DT[dtype], device="cuda")
+    fp4 = torch.empty((B, S, D // 2), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((B, S, D // 16), dtype=torch.uint8, device="cuda")
+    ops.csa_compress(a.cuda(), b.cuda(), z.cuda(), m, out=out, out_fp4=fp4, out_sf=sf, gscale=1.0)
+    ref = oracle.csa_compress(a, b, z, m)
+    _assert_close(_np(out), oracle.round_out(ref, dtype) if dtype == "bf16" else ref, dtype)
+    # the NVFP4 output is the exact quantisation of the stored entries
+    q = oracle.nvfp4_quantize(out.cpu(), 1.0)
+    np.testing.assert_array_equal(sf.cpu().numpy(), q["sf"])
+    got = fp4.cpu().numpy()
+    canon = lambda c: np.where(c == 8, 0, c)
+    np.testing.assert_array_equal(canon(got & 0xF), canon(q["codes"][..., 0::2]))
+    np.testing.assert_array_equal(canon(got >> 4), canon(q["codes"][..., 1::2]))
+
+
+def test_csa_compress_decode_window(ops):
+    """Decode mode: rings of 2m raw rows, entry emitted only when (p+1) % m == 0."""
+    m, D, B = 4, 128, 3
+    T = 64
+    a, b, z = (_randn((B, T, D), "bf16", s) for s in (6, 7, 8))
+    ref = oracle.round_out(oracle.csa_compress(a, b, z, m), "bf16")
+    cap = T // m
+    out = torch.zeros((B, cap, D), dtype=torch.bfloat16, device="cuda")
+    ring = {n: torch.zeros((B, 2 * m, D), dtype=torch.bfloat16, device="cuda") for n in "abz"}
+    pos = torch.zeros((B,), dtype=torch.int32, device="cuda")
+    src = {"a": a.cuda(), "b": b.cuda(), "z": z.cuda()}
+    for p in range(T):
+        for n in "abz":
+            ops.csa_ring_append(src[n][:, p].contiguous(), ring[n], pos)
+        ops.csa_compress(ring["a"], ring["b"], ring["z"], m, out=out, ring_pos=pos, out_bstride=cap)
+        ops.csa_pos_advance(pos, 1)
+    _assert_close(_np(out), ref, "bf16")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_hca_compress(ops, dtype):
+    B, T, D, m = 2, 128 * 9 + 50, 128, 128
+    a = _randn((B, T, D), dtype, 9)
+    z = _randn((B, T, D), dtype, 10, np.sqrt(2.0))
+    out = torch.empty((B, T // m, D), dtype=DT[dtype], device="cuda")
+    ops.hca_compress(a.cuda(), z.cuda(), m, out)
+    ref = oracle.hca_compress(a, z, m)
+    _assert_close(_np(out), oracle.round_out(ref, dtype) if dtype == "bf16" else ref, dtype)
+
+
+# ---------------------------------------------------------------- indexer
+
+def _quant_inputs(ops, B, T, S, HI, DI, seed):
+    qi = _randn((B, T, HI, DI), "bf16", seed)
+    ki = _randn((B, S, DI), "bf16", seed + 1)
+    q4 = torch.empty((B, T, HI, DI // 2), dtype=torch.uint8, device="cuda")
+    qs = torch.empty((B, T, HI, DI // 16), dtype=torch.uint8, device="cuda")
+    k4 = torch.empty((B, S, DI // 2), dtype=torch.uint8, device="cuda")
+    ks = torch.empty((B, S, DI // 16), dtype=torch.uint8, device="cuda")
+    ops.nvfp4_quantize(qi.cuda(), q4, qs)
+    ops.nvfp4_quantize(ki.cuda(), k4, ks)
+    return qi, ki, q4, qs, k4, ks
+
+
+@pytest.mark.parametrize("HI,DI,sdt", [(4, 64, "bf16"), (2, 32, "f32"), (4, 64, "f32"), (1, 64, "bf16"),
+                                       (8, 64, "bf16")])
+def test_indexer_score(ops, HI, DI, sdt):
+    B, T, m = 2, 700, 4
+    S = T // m
+    qi, ki, q4, qs, k4, ks = _quant_inputs(ops, B, T, S, HI, DI, 11)
+    w = torch.rand((B, T, HI), generator=torch.Generator().manual_seed(3))
+    pos0 = torch.tensor([0, 37], dtype=torch.int32)
+    score = torch.full((B, T, S), float("nan"), dtype=DT[sdt], device="cuda")
+    ops.indexer_score(q4, qs, k4, ks, w.cuda(), pos0.cuda(), score, S, m)
+    qhat = oracle.nvfp4_quantize(qi)["xhat"]
+    khat = oracle.nvfp4_quantize(ki)["xhat"]
+    pos = np.arange(T)[None] + pos0.numpy()[:, None]
+    ref = oracle.indexer_score(qhat, khat, w, pos, m)
+    got = _np(score)
+    vis = ~np.isnan(ref)
+    assert np.all(~np.isnan(got[vis]))
+    if sdt == "f32":
+        np.testing.assert_allclose(got[vis], ref[vis], rtol=2e-6, atol=1e-6)
+    else:
+        _assert_close(got[vis], formats.bf16(ref[vis]), "bf16")
+    # the invisible region is left unwritten (still NaN)
+    assert np.all(np.isnan(got[~vis]))
+
+
+def test_indexer_score_row_chunks(ops):
+    """Chunked rows (row0 > 0) and a chunk that is not a multiple of the token tile."""
+    B, T, S, HI, DI, m = 1, 1000, 250, 4, 64, 4
+    qi, ki, q4, qs, k4, ks = _quant_inputs(ops, B, T, S, HI, DI, 21)
+    w = torch.rand((B, T, HI), generator=torch.Generator().manual_seed(5)).cuda()
+    pos0 = torch.zeros((B,), dtype=torch.int32, device="cuda")
+    full = torch.zeros((B, T, S), dtype=torch.float32, device="cuda")
+    ops.indexer_score(q4, qs, k4, ks, w, pos0, full, S, m)
+    for r0, tc in ((0, 333), (333, 333), (666, 334)):
+        part = torch.zeros((B, tc, S), dtype=torch.float32, device="cuda")
+        ops.indexer_score(q4, qs, k4, ks, w, pos0, part, S, m, row0=r0, T_chunk=tc)
+        torch.testing.assert_close(part, full[:, r0:r0 + tc], rtol=0, atol=0)
+
+
+# ------------------------------------------------------------------ top-k
+
+@pytest.mark.parametrize("sdt", ["f32", "bf16"])
+@pytest.mark.parametrize("k", [1, 7, 64, 512])
+def test_topk_bit_exact(ops, sdt, k):
+    B, T, m = 2, 600, 4
+    S = 9000 // m if k == 512 else T // m
+    T = max(T, S * m)
+    g = torch.Generator().manual_seed(k)
+    sc = torch.randn((B, T, S), generator=g)
+    # ties and zeros: quantise a third of the rows coarsely, add +-0
+    sc[:, ::3] = torch.round(sc[:, ::3] * 2) / 2
+    sc[:, 1::5] = torch.relu(sc[:, 1::5])
+    sc[0, 10, :50] = -0.0
+    sc = sc.to(DT[sdt])
+    pos0 = torch.tensor([0, 3], dtype=torch.int32)
+    idx = torch.empty((B, T, k), dtype=torch.int32, device="cuda")
+    ops.topk_select(sc.cuda(), idx, S, m, pos0.cuda())
+    pos = np.arange(T)[None] + pos0.numpy()[:, None]
+    ref = oracle.topk_select(_np(sc), pos, m, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+
+
+def test_topk_long_rows_all_equal(ops):
+    """A row of identical scores: the k smallest indices."""
+    S, k = 20000, 300
+    sc = torch.zeros((1, 1, S), dtype=torch.bfloat16, device="cuda")
+    pos0 = torch.tensor([4 * S], dtype=torch.int32, device="cuda")
+    idx = torch.empty((1, 1, k), dtype=torch.int32, device="cuda")
+    ops.topk_select(sc, idx, S, 4, pos0)
+    np.testing.assert_array_equal(idx.cpu().numpy()[0, 0], np.arange(k))
+
+
+# -------------------------------------------------------------- attention
+
+def _attn_inputs(B, T, H, D, S, dtype, seed, q_scale=1.0):
+    q = _randn((B, T, H, D), dtype, seed, q_scale)
+    kv_c = _randn((B, S, D), dtype, seed + 1)
+    raw = _randn((B, T, D), dtype, seed + 2)
+    sink = torch.randn((H,), generator=torch.Generator().manual_seed(seed + 3))
+    return q, kv_c, raw, sink
+
+
+def _attn_tol(dtype):
+    return (lambda g, r: np.testing.assert_allclose(g, r, rtol=1e-5, atol=1e-5)) if dtype == "f32" else \
+        (lambda g, r: np.testing.assert_allclose(g, r, rtol=0, atol=2e-2))
+
+
+@pytest.mark.parametrize("dtype,H,D", [("f32", 8, 64), ("bf16", 64, 128), ("bf16", 128, 128), ("bf16", 16, 64)])
+def test_sparse_attn(ops, dtype, H, D):
+    B, T, m, k, W = 2, 300, 4, 24, 128
+    S = T // m
+    tau = 1.0 / np.sqrt(D)
+    q, kv_c, raw, sink = _attn_inputs(B, T, H, D, S, dtype, 30)
+    pos0 = torch.tensor([0, 5], dtype=torch.int32)
+    pos = np.arange(T)[None] + pos0.numpy()[:, None]
+    idx = oracle.topk_select(np.random.default_rng(0).standard_normal((B, T, S)), pos, m, k)
+    idx_t = torch.from_numpy(idx)
+    out = torch.empty_like(q, device="cuda")
+    lse = torch.empty((B, T, H), dtype=torch.float32, device="cuda")
+    ops.sparse_attn_fwd(q.cuda(), kv_c.cuda(), idx_t.cuda(), raw.cuda(), sink.cuda(), tau, W, pos0.cuda(), out,
+                        lse)
+    ro, rl = oracle.sparse_attn(q, kv_c, idx, raw, T, sink, tau, W, pos)
+    _attn_tol(dtype)(_np(out), oracle.round_out(ro, dtype))
+    np.testing.assert_allclose(lse.cpu().numpy(), rl, rtol=1e-5 if dtype == "f32" else 2e-3, atol=1e-4)
+
+
+@pytest.mark.parametrize("dtype,H,D,m", [("f32", 8, 64, 4), ("bf16", 64, 128, 16), ("bf16", 128, 128, 32)])
+def test_hca_dense_attn(ops, dtype, H, D, m):
+    B, T, W = 2, 700, 128
+    S = T // m
+    tau = 1.0 / np.sqrt(D)
+    q, kv_c, raw, sink = _attn_inputs(B, T, H, D, S, dtype, 40)
+    pos0 = torch.tensor([0, 9], dtype=torch.int32)
+    pos = np.arange(T)[None] + pos0.numpy()[:, None]
+    out = torch.empty_like(q, device="cuda")
+    ops.hca_dense_attn_fwd(q.cuda(), kv_c.cuda(), raw.cuda(), sink.cuda(), tau, W, pos0.cuda(), out, m)
+    ro, _ = oracle.dense_attn(q, kv_c, raw, T, sink, tau, W, pos, m)
+    _attn_tol(dtype)(_np(out), oracle.round_out(ro, dtype))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_split_path_merge_equals_fused(ops, dtype):
+    """sparse_attn_fwd(W=0, no sink) -> (o_c, lse_c), then swa_sink_merge, equals
+    the fused call; both equal the oracle."""
+    B, T, H, D, m, k, W = 1, 260, 16, 64, 4, 16, 128
+    S = T // m
+    tau = 0.125
+    q, kv_c, raw, sink = _attn_inputs(B, T, H, D, S, dtype, 50)
+    pos0 = torch.zeros((B,), dtype=torch.int32)
+    pos = np.arange(T)[None]
+    idx = oracle.topk_select(np.random.default_rng(1).standard_normal((B, T, S)), pos, m, k)
+    dq, dkv, draw, dsink, didx = q.cuda(), kv_c.cuda(), raw.cuda(), sink.cuda(), torch.from_numpy(idx).cuda()
+    oc = torch.empty_like(dq)
+    lc = torch.empty((B, T, H), dtype=torch.float32, device="cuda")
+    ops.sparse_attn_fwd(dq, dkv, didx, draw, None, tau, 0, pos0.cuda(), oc, lc)
+    merged = torch.empty_like(dq)
+    ops.swa_sink_merge(oc, lc, dq, draw, dsink, tau, W, pos0.cuda(), merged)
+    ro, _ = oracle.sparse_attn(q, kv_c, idx, raw, T, sink, tau, W, pos)
+    _attn_tol(dtype)(_np(merged), oracle.round_out(ro, dtype))
+
+
+def test_ring_window_decode_positions(ops):
+    """raw_cap < T: the window reads slot j % raw_cap (a decode ring)."""
+    B, H, D, cap, W, m = 2, 64, 128, 128, 128, 4
+    p0 = np.array([5000, 777])
+    S = 2000
+    q = _randn((B, 1, H, D), "bf16", 60)
+    kv_c = _randn((B, S, D), "bf16", 61)
+    ring = _randn((B, cap, D), "bf16", 62)
+    sink = torch.randn((H,), generator=torch.Generator().manual_seed(63))
+    idx = np.sort(np.random.default_rng(2).choice(S, size=(B, 1, 64), replace=False), axis=-1).astype(np.int32)
+    idx[1, 0, 60:] = -1
+    out = torch.empty((B, 1, H, D), dtype=torch.bfloat16, device="cuda")
+    pos0 = torch.from_numpy(p0.astype(np.int32)).cuda()
+    ops.sparse_attn_fwd(q.cuda(), kv_c.cuda(), torch.from_numpy(idx).cuda(), ring.cuda(), sink.cuda(),
+                        1 / np.sqrt(D), W, pos0, out, raw_cap=cap)
+    ro, _ = oracle.sparse_attn(q, kv_c, idx, ring, cap, sink, 1 / np.sqrt(D), W, p0[:, None])
+    _attn_tol("bf16")(_np(out), oracle.round_out(ro, "bf16"))
+
+
+def test_no_device_timeouts(ops):
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
