@@ -255,9 +255,10 @@ def _attn_tol(dtype):
         (lambda g, r: np.testing.assert_allclose(g, r, rtol=0, atol=2e-2))
 
 
-@pytest.mark.parametrize("dtype,H,D", [("f32", 8, 64), ("bf16", 64, 128), ("bf16", 128, 128), ("bf16", 16, 64)])
-def test_sparse_attn(ops, dtype, H, D):
-    B, T, m, k, W = 2, 300, 4, 24, 128
+@pytest.mark.parametrize("dtype,H,D,k", [("f32", 8, 64, 24), ("bf16", 64, 128, 24), ("bf16", 128, 128, 24),
+                                         ("bf16", 64, 128, 200), ("bf16", 128, 128, 300)])
+def test_sparse_attn(ops, dtype, H, D, k):
+    B, T, m, W = 2, 1300, 4, 128
     S = T // m
     tau = 1.0 / np.sqrt(D)
     q, kv_c, raw, sink = _attn_inputs(B, T, H, D, S, dtype, 30)
@@ -274,7 +275,8 @@ def test_sparse_attn(ops, dtype, H, D):
     np.testing.assert_allclose(lse.cpu().numpy(), rl, rtol=1e-5 if dtype == "f32" else 2e-3, atol=1e-4)
 
 
-@pytest.mark.parametrize("dtype,H,D,m", [("f32", 8, 64, 4), ("bf16", 64, 128, 16), ("bf16", 128, 128, 32)])
+@pytest.mark.parametrize("dtype,H,D,m", [("f32", 8, 64, 4), ("bf16", 64, 128, 16), ("bf16", 128, 128, 32),
+                                         ("bf16", 16, 128, 4), ("bf16", 32, 128, 128), ("bf16", 64, 128, 128)])
 def test_hca_dense_attn(ops, dtype, H, D, m):
     B, T, W = 2, 700, 128
     S = T // m
@@ -288,11 +290,11 @@ def test_hca_dense_attn(ops, dtype, H, D, m):
     _attn_tol(dtype)(_np(out), oracle.round_out(ro, dtype))
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_split_path_merge_equals_fused(ops, dtype):
+@pytest.mark.parametrize("dtype,H,D", [("f32", 16, 64), ("bf16", 64, 128)])
+def test_split_path_merge_equals_fused(ops, dtype, H, D):
     """sparse_attn_fwd(W=0, no sink) -> (o_c, lse_c), then swa_sink_merge, equals
     the fused call; both equal the oracle."""
-    B, T, H, D, m, k, W = 1, 260, 16, 64, 4, 16, 128
+    B, T, m, k, W = 1, 260, 4, 16, 128
     S = T // m
     tau = 0.125
     q, kv_c, raw, sink = _attn_inputs(B, T, H, D, S, dtype, 50)
@@ -326,6 +328,61 @@ def test_ring_window_decode_positions(ops):
                         1 / np.sqrt(D), W, pos0, out, raw_cap=cap)
     ro, _ = oracle.sparse_attn(q, kv_c, idx, ring, cap, sink, 1 / np.sqrt(D), W, p0[:, None])
     _attn_tol("bf16")(_np(out), oracle.round_out(ro, "bf16"))
+
+
+def test_attn_rescale_path(ops):
+    """Later KV tiles with far larger logits force the running-max rescale of the
+    O^T accumulator and row sums (tiles ordered: entries, then the window)."""
+    B, T, H, D, m, k, W = 1, 600, 64, 128, 4, 150, 128
+    S = T // m
+    q = _randn((B, T, H, D), "bf16", 70)
+    kv_c = _randn((B, S, D), "bf16", 71, 0.05)          # small entries: small logits
+    raw = _randn((B, T, D), "bf16", 72, 6.0)            # window rows: logits ~ x100
+    sink = torch.randn((H,), generator=torch.Generator().manual_seed(73))
+    pos0 = torch.zeros((B,), dtype=torch.int32)
+    pos = np.arange(T)[None]
+    idx = oracle.topk_select(np.random.default_rng(3).standard_normal((B, T, S)), pos, m, k)
+    out = torch.empty_like(q, device="cuda")
+    lse = torch.empty((B, T, H), dtype=torch.float32, device="cuda")
+    ops.sparse_attn_fwd(q.cuda(), kv_c.cuda(), torch.from_numpy(idx).cuda(), raw.cuda(), sink.cuda(),
+                        1 / np.sqrt(D), W, pos0.cuda(), out, lse)
+    ro, rl = oracle.sparse_attn(q, kv_c, idx, raw, T, sink, 1 / np.sqrt(D), W, pos)
+    _attn_tol("bf16")(_np(out), oracle.round_out(ro, "bf16"))
+    np.testing.assert_allclose(lse.cpu().numpy(), rl, rtol=2e-3, atol=1e-3)
+
+
+def test_attn_row_chunks_and_empty_sets(ops):
+    """row0 > 0 chunks write only their rows; W = 0 rows with no entry give 0."""
+    B, T, H, D, m, k, W = 1, 700, 64, 128, 4, 64, 128
+    S = T // m
+    q, kv_c, raw, sink = _attn_inputs(B, T, H, D, S, "bf16", 80)
+    pos0 = torch.zeros((B,), dtype=torch.int32, device="cuda")
+    pos = np.arange(T)[None]
+    idx = oracle.topk_select(np.random.default_rng(4).standard_normal((B, T, S)), pos, m, k)
+    dq, dkv, draw, dsink = q.cuda(), kv_c.cuda(), raw.cuda(), sink.cuda()
+    full = torch.empty_like(dq)
+    ops.sparse_attn_fwd(dq, dkv, torch.from_numpy(idx).cuda(), draw, dsink, 1 / np.sqrt(D), W, pos0, full)
+    part = torch.zeros_like(dq)
+    for r0, tc in ((0, 250), (250, 250), (500, 200)):
+        ops.sparse_attn_fwd(dq, dkv, torch.from_numpy(idx[:, r0:r0 + tc].copy()).cuda(), draw, dsink,
+                            1 / np.sqrt(D), W, pos0, part, row0=r0, T_chunk=tc)
+    torch.testing.assert_close(part, full, rtol=0, atol=0)
+    # no window, no entries for the first m-1 rows: output 0, lse -inf
+    o0 = torch.full_like(dq, 7.0)
+    l0 = torch.zeros((B, T, H), dtype=torch.float32, device="cuda")
+    ops.sparse_attn_fwd(dq, dkv, torch.from_numpy(idx).cuda(), draw, None, 1 / np.sqrt(D), 0, pos0, o0, l0)
+    assert torch.all(o0[:, : m - 1] == 0) and torch.all(torch.isinf(l0[:, : m - 1]))
+    ro, _ = oracle.sparse_attn(q, kv_c, idx, raw, T, None, 1 / np.sqrt(D), 0, pos)
+    _attn_tol("bf16")(_np(o0), oracle.round_out(ro, "bf16"))
+
+
+def test_attn_unsupported_shapes_rejected(ops):
+    q = torch.zeros((1, 8, 16, 64), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((1, 2, 64), dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros((1, 8, 2), dtype=torch.int32, device="cuda")
+    pos0 = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    with pytest.raises(ops.CsaError):
+        ops.sparse_attn_fwd(q, kv, idx, kv, None, 1.0, 0, pos0, torch.empty_like(q))
 
 
 def test_no_device_timeouts(ops):
