@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark: one CSA prefill layer (T = 32768, 64 heads x dim 128, MQA KV dim 128,
+4:1 overlapping compression -> 8192 entries, NVFP4 indexer 4 x 64, top-k 512,
+raw window 128, sink) per step, on synthetic seeded inputs.
+
+One JSON line on rank 0:
+  value      tokens/s of the whole job (inputs resident in HBM), max over ranks
+  e2e        the same through the C ABI with host buffers: pinned H2D of every
+             input, the layer, D2H of the output, all inside the timed region
+  roofline   the dominant kernel (sparse_attn_fwd, tensor-bound): algorithmic
+             FLOPs per launch / its CUDA-event duration inside the timed region,
+             against the measured bf16 peak
+  kernels    per-kernel average duration (ms) and algorithmic rate
+  cpu_baseline  the CPU oracle on a bounded sample of the same workload
+
+--impl reference times the CPU oracle as the reference arm (rank 0 only).
+Multi-GPU (torchrun): every rank runs its own independent layer (weak scaling,
+no collective on the data path; the timing uses a MAX all-reduce).
+"""
+from __future__ import annotations
+
+import argparse
+import contextlib
+import datetime
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA/HCA attn-layer prefill tokens/s & 1M-ctx decode steps/s; % of roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--chunk", type=int, default=0, help="query rows per indexer/top-k chunk (0 = all)")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-rows", type=int, default=96, help="query rows in the CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--T", type=int, default=0,
+                    help="profiling case: override the layer's token count (not a bench line)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def algorithmic_work(cfg):
+    """Per-layer algorithmic work of each step (definitions in the design notes)."""
+    T, H, D, m, k, W, S = cfg.T, cfg.H, cfg.D, cfg.m, cfg.k, cfg.W, cfg.S
+    HI, DI = cfg.HI, cfg.DI
+    rows = sel = vis_pairs = 0
+    for t in range(T):
+        vis = min(S, (t + 1) // m)
+        vis_pairs += vis
+        sel += min(k, vis) + min(W, t + 1)
+    B = cfg.B
+    esz = 2
+    return {
+        "attn_flops": B * 4.0 * H * D * sel,
+        "attn_rows": B * sel,
+        "indexer_pairs": B * vis_pairs,
+        "indexer_flops": B * 2.0 * vis_pairs * HI * DI,
+        "indexer_bytes": B * (vis_pairs * esz + T * HI * (DI // 2 + DI // 16 + 4) + S * (DI // 2 + DI // 16)),
+        "topk_bytes": B * (vis_pairs * esz + T * k * 4),
+        "compress_bytes": B * (3 * T * D * esz + S * D * esz),
+        "compress_keys_bytes": B * (3 * T * DI * esz + S * (DI // 2 + DI // 16)),
+        "quant_bytes": B * (T * HI * DI * esz + T * HI * (DI // 2 + DI // 16)),
+        "attn_hbm_bytes": B * (2 * T * H * D * esz + T * k * 4),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.4)
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        samples = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    samples.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        inside = [s for s in samples if t0 - 0.05 <= s[0] <= t1 + 0.05] or samples[-3:]
+        if not inside:
+            return None
+        mhz = sorted(s[1] for s in inside)
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for s in inside for i, v in enumerate(s[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": max(s[2] for s in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+class OracleSample:
+    """The CPU oracle as it stands, timed on a bounded sample of the layer:
+    the compressors + NVFP4 quantisation once over all T tokens, then
+    indexer/top-k/attention on batches of query rows (uniform, seed 1234);
+    throughput = T / (t_compress + t_per_row * T)."""
+
+    def __init__(self, cfg):
+        import numpy as np
+        import oracle
+        from long_context_compressed_compress_b200 import inputs
+        self.np, self.oracle, self.cfg = np, oracle, cfg
+        # host inputs converted to float64 once (the oracle's working precision)
+        self.x = {k: v.to(torch_f64()).numpy() for k, v in inputs.layer_inputs(cfg, device="cpu").items()}
+        self.idx = np.full((cfg.B, cfg.T, cfg.k), -1, dtype=np.int32)
+        self.pos = np.arange(cfg.T)[None]
+        self.rng = np.random.default_rng(1234)
+        try:
+            from threadpoolctl import threadpool_info
+            self.cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        except Exception:  # pragma: no cover
+            self.cores = 1
+        c, x = cfg, self.x
+        t0 = time.perf_counter()
+        self.kv = oracle.round_out(oracle.csa_compress(x["a"], x["b"], x["z"], c.m), c.dtype)
+        ks = oracle.round_out(oracle.csa_compress(x["a_I"], x["b_I"], x["z_I"], c.m), c.dtype)
+        self.khat = oracle.nvfp4_quantize(ks)["xhat"]
+        self.qhat = oracle.nvfp4_quantize(x["q_I"])["xhat"]
+        self.t_comp = time.perf_counter() - t0
+        self.t_rows = 0.0
+        self.n_rows = 0
+
+    def rows(self, n):
+        np, o, c, x = self.np, self.oracle, self.cfg, self.x
+        ts = self.rng.integers(0, c.T, size=n)
+        t0 = time.perf_counter()
+        for t in ts:
+            t = int(t)
+            pos = np.array([[t]])
+            sc = o.round_scores(o.indexer_score(self.qhat[:, t:t + 1], self.khat, x["w"][:, t:t + 1], pos, c.m),
+                                "bf16" if c.dtype != "f32" else "f32")
+            idx = o.topk_select(sc, pos, c.m, c.k)
+            self.idx[0, t] = idx[0, 0]
+            o.sparse_attn(x["q"], self.kv, self.idx, x["kv_raw"], c.T, x["sink"], c.tau, c.W, self.pos,
+                          rows=[(0, t)])
+        dt = time.perf_counter() - t0
+        self.t_rows += dt
+        self.n_rows += n
+        return dt
+
+    def value(self):
+        per_row = self.t_rows / max(1, self.n_rows)
+        return self.cfg.B * self.cfg.T / (self.t_comp + per_row * self.cfg.B * self.cfg.T)
+
+    def describe(self):
+        return {"value": self.value(), "unit": "tokens/s", "cores": self.cores, "kind": "oracle",
+                "sample": f"compressors + NVFP4 over all {self.cfg.T} tokens ({self.t_comp:.1f} s), then "
+                          f"indexer/top-k/attention on {self.n_rows} uniform query rows "
+                          f"({self.t_rows:.1f} s), extrapolated to {self.cfg.T} rows"}
+
+
+def torch_f64():
+    import torch
+    return torch.float64
+
+
+def cpu_baseline(cfg, n_rows):
+    s = OracleSample(cfg)
+    s.rows(n_rows)
+    return s.describe()
+
+
+def run_reference(args, cfg, rank):
+    """Reference arm: the CPU oracle, each step a bounded sample of query rows."""
+    if rank != 0:
+        return
+    per_step = 4
+    s = OracleSample(cfg)
+    for _ in range(args.warmup):
+        s.rows(1)
+    s.t_rows, s.n_rows = 0.0, 0
+    for _ in range(args.steps):
+        s.rows(per_step)
+    v = s.value()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": cfg.B * cfg.T / v * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) inputs, U(0,1) indexer weights, N(0,1) sink)",
+        "config": {"workload": "csa_prefill_32k" if not args.T else f"csa_prefill_T{cfg.T}", "B": cfg.B, "T": cfg.T, "H": cfg.H, "D": cfg.D, "m": cfg.m,
+                   "S": cfg.S, "k": cfg.k, "HI": cfg.HI, "DI": cfg.DI, "W": cfg.W},
+        "cpu_baseline": s.describe(),
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from long_context_compressed_compress_b200 import configs
+    cfg = configs.CSA_PREFILL
+    if args.T:
+        cfg = configs.scaled(cfg, T=args.T)
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import build
+    build.build()
+    from long_context_compressed_compress_b200 import inputs, layer
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    peaks = load_peaks()
+    work = algorithmic_work(cfg)
+    x = inputs.layer_inputs(cfg, device="cuda")
+    lay = layer.CsaPrefill(cfg, chunk=args.chunk or None)
+    stream = torch.cuda.current_stream()
+
+    # per-kernel CUDA events on the launching stream, inside the timed region
+    ev = {}
+
+    @contextlib.contextmanager
+    def timer(name):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        yield
+        e1.record(stream)
+        ev.setdefault(name, []).append((e0, e1))
+
+    for _ in range(args.warmup):
+        lay.run(x)
+    torch.cuda.synchronize()
+    ev.clear()
+
+    gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid) if hasattr(
+        torch.cuda.get_device_properties(dev), "uuid") else str(local)
+    sampler = ClockSampler(gpu_uuid)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(args.steps):
+        lay.run(x, timer=timer)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    ms_total = s0.elapsed_time(s1)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    kern = {}
+    for name, lst in ev.items():
+        kern[name] = sum(a.elapsed_time(b) for a, b in lst) / args.steps
+    launches = lay.launches * args.steps
+
+    # ---- end to end through the C ABI with host buffers
+    host = {k: v.to("cpu").pin_memory() for k, v in x.items()}
+    out_host = torch.empty(lay.out.shape, dtype=lay.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    xd = {k: torch.empty_like(v) for k, v in x.items()}
+    for _ in range(2 if args.e2e_steps else 0):
+        for k2, v in host.items():
+            xd[k2].copy_(v, non_blocking=True)
+        lay.run(xd)
+        out_host.copy_(lay.out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for k2, v in host.items():
+            xd[k2].copy_(v, non_blocking=True)
+        lay.run(xd)
+        out_host.copy_(lay.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / max(1, args.e2e_steps)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    tokens = cfg.B * cfg.T
+    value = world * tokens / (ms_step * 1e-3)
+    attn_ms = kern.get("sparse_attn_fwd", float("nan"))
+    achieved = work["attn_flops"] / (attn_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "sparse_attn_fwd_csa_prefill_32k.json")
+    if os.path.exists(prof):
+        with open(prof) as f:
+            pj = json.load(f)
+        if pj.get("kernel_hash") == kernel_hash():
+            traffic = pj.get("dram_bytes_per_launch")
+    rates = {
+        "csa_compress": ("GB/s", work["compress_bytes"]),
+        "csa_compress_indexer_keys": ("GB/s", work["compress_keys_bytes"]),
+        "nvfp4_quantize": ("GB/s", work["quant_bytes"]),
+        "indexer_score": ("GB/s", work["indexer_bytes"]),
+        "topk_select": ("GB/s", work["topk_bytes"]),
+        "sparse_attn_fwd": ("TFLOP/s", work["attn_flops"]),
+    }
+    kernels = {}
+    for name, t in kern.items():
+        unit, amount = rates.get(name, ("", 0))
+        rate = amount / (t * 1e-3) / (1e9 if unit == "GB/s" else 1e12) if t > 0 else None
+        pk = peaks["hbm_gbs"] if unit == "GB/s" else peak
+        kernels[name] = {"ms": round(t, 5), "achieved": rate and round(rate, 2), "unit": unit,
+                         "frac": rate and round(rate / pk, 4)}
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs, U(0,1) indexer weights, N(0,1) sink)",
+        "config": {"workload": "csa_prefill_32k", "B": cfg.B, "T": cfg.T, "H": cfg.H, "D": cfg.D, "m": cfg.m,
+                   "S": cfg.S, "k": cfg.k, "HI": cfg.HI, "DI": cfg.DI, "W": cfg.W,
+                   "chunk": lay.chunk, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (q + out = 1.07 GB per step)"},
+        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "roofline": {"bound": "tensor", "kernel": "sparse_attn_fwd", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                     "algorithmic_flops_per_launch": work["attn_flops"]},
+        "kernels": kernels,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def kernel_hash():
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("attn_tc.cu", "common.cuh", "attention.cu"):
+        with open(os.path.join(ROOT, "long_context_compressed_compress_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+if __name__ == "__main__":
+    main()

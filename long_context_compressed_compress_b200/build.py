@@ -43,16 +43,19 @@ def up_to_date() -> bool:
     return os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime()
 
 
-def build(verbose: bool = False, force: bool = False, extra_flags=None) -> str:
-    if not force and up_to_date():
+def build(verbose: bool = False, force: bool = False, extra_flags=None, lib_path=None, build_dir=None) -> str:
+    """Compile csrc/*.cu and link ``lib_path`` (default: the in-tree library)."""
+    lib = lib_path or LIB
+    bdir = build_dir or BUILD
+    if not force and lib_path is None and up_to_date():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    os.makedirs(bdir, exist_ok=True)
     nvcc = _nvcc()
     flags = NVCC_FLAGS + list(extra_flags or [])
     objs = []
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         cmd = [nvcc, *flags, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -65,13 +68,13 @@ def build(verbose: bool = False, force: bool = False, extra_flags=None) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, sources()))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

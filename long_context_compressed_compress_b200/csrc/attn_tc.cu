@@ -13,9 +13,13 @@
 // (full tcgen05 rate) where the transposed form would need M = 64.
 //
 // Roles (one CTA per SM, persistent over work units):
-//   producer warps (2): gather the unit's KV rows (top-k entries or every
-//     visible entry, then the raw-window tokens) into 128-row tiles with
-//     cp.async in the 128-byte-swizzled layout; load Q.
+//   producer warp (1): gathers the unit's KV rows (top-k entries or every
+//     visible entry, then the raw-window tokens) into 128-row tiles with TMA
+//     tile::gather4 (four rows per instruction, one 4-row group per lane, the
+//     128-byte swizzle applied by the TMA unit); Q arrives by a 2D TMA load.
+//     Completion is tracked by mbarrier transaction bytes.  The compressed
+//     part of the row list is padded to a multiple of 4 rows (masked rows,
+//     zero-filled by out-of-range coordinates) so a group never mixes sources.
 //   MMA warp (1): issues QK(i+1) before PV(i) so the tensor core works on the
 //     next tile while the softmax runs.
 //   softmax warpgroups (N/64, 4 warps each): thread = TMEM lane = KV row of S^T
@@ -26,7 +30,29 @@
 //     bf16 (MN-major, swizzled) for the PV MMA.
 // All waits are bounded; a wait that gives up sets the device status word and
 // an abort flag that every role polls, so the kernel always returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
+
+// Compile-time event trace for pipeline analysis (debug builds only):
+// globaltimer stamps of each role's per-tile events in CTA 0.
+#ifdef CSA_TRACE
+__device__ unsigned long long* g_csa_trace;
+#define CSA_TR(unit, tile, ev)                                                                   \
+  do {                                                                                           \
+    if (blockIdx.x == 0 && g_csa_trace != nullptr && (unit) < 64 && (tile) < 16) {               \
+      unsigned long long t_;                                                                     \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                     \
+      g_csa_trace[((unit) * 16 + (tile)) * 8 + (ev)] = t_;                                        \
+    }                                                                                            \
+  } while (0)
+extern "C" int csa_debug_set_trace(void* p) {
+  return cudaMemcpyToSymbol(g_csa_trace, &p, sizeof(p)) == cudaSuccess ? 0 : 4;
+}
+#else
+#define CSA_TR(unit, tile, ev) do { } while (0)
+#endif
 
 namespace csa {
 
@@ -39,19 +65,32 @@ struct TcCfg {
   static constexpr int N = 64 * NB;                       // MMA N (token, head) columns
   static constexpr int kGroups = N / 32;                  // softmax warpgroups
   static constexpr int kSoftWarps = 4 * kGroups;
-  static constexpr int kProdWarps = NB == 1 ? 2 : 1;
+  static constexpr int kProdWarps = NB == 1 ? 4 : 2;   // gather issue rate scales with warps
   static constexpr int kThreads = 32 * (kSoftWarps + kProdWarps + 1);
   static constexpr int kStages = NB == 1 ? 4 : 2;
   static constexpr int kQBytes = N * kTcDim * 2;
   static constexpr int kKVBytes = kTcTile * kTcDim * 2;   // 32 KB
   static constexpr int kPBytes = kTcTile * N * 2;
-  static constexpr uint32_t kTmemCols = 4 * N;            // S x2, O x2
+  // N = 64: the per-column row sums come from a second PV-shaped MMA with an
+  // all-ones A operand (L^T += 1 . P^T) into TMEM; N = 128 keeps them in registers
+  static constexpr bool kSumMma = NB == 1;
+  static constexpr uint32_t kTmemCols = kSumMma ? 512 : 4 * N;   // S x2, O x2 (+ L x2)
+  static constexpr int kOnesBytes = kSumMma ? kTcTile * 128 : 1024;
 };
 
 struct TcUnit {
   int b, r0, ntok, n_c, n_w, jlo, p0, nt;
   int n_all;   // leading rows valid for every token of the unit
+  int n_cp;    // n_c rounded up to 4: window rows start here
 };
+
+struct TcMaps {
+  CUtensorMap q;     // [B*Tq*H, 128] bf16, box 64 x H (one token)
+  CUtensorMap kv;    // [B*kv_bstride, 128] bf16, box 64 x 128 (one tile half)
+  CUtensorMap raw;   // [B*raw_cap, 128] bf16, box 64 x 128 (one tile half)
+};
+
+constexpr int kTcMaxIdxTiles = 8;   // top-k up to 1024 entries per query
 
 template <int NB>
 struct __align__(1024) TcSmem {
@@ -59,11 +98,14 @@ struct __align__(1024) TcSmem {
   uint8_t q[2][C::kQBytes];
   uint8_t kv[C::kStages][C::kKVBytes];
   uint8_t p[2][C::kPBytes];
+  uint8_t ones[C::kOnesBytes];   // bf16 1.0 (A operand of the row-sum MMA)
   uint64_t kv_full[C::kStages], kv_empty[C::kStages];
   uint64_t q_full[2], q_empty[2], s_full[2], s_free[2], p_full[2], p_empty[2], o_full[2], o_empty[2];
   float xch[2 * NB][4][32];
   float mcol[2 * NB][32];
   float alpha[2 * NB][32];
+  float dlt[2 * NB][32];
+  float sink_l2[128];      // sink logits in log2 units (-inf without a sink)
   TcUnit info[2];
   uint32_t tmem;
   int abort_flag;
@@ -86,17 +128,25 @@ struct TcArgs {
   int sparse;            // 1: CSA (idx), 0: HCA (all visible entries)
   int units_per_b;
   int n_units;
+  int kv_rows, raw_rows; // rows of the kv / raw tensor maps (an index equal to them is out of range)
 };
 
-__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
-  for (long long i = 0; i < kWaitLimit; ++i) {
+// Time-bounded wait shared by every role: returns false at once when another
+// role has aborted, and aborts the CTA (recording the wait site) after kWaitNs.
+__device__ __forceinline__ bool tc_wait_site(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag,
+                                             int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 255 && *abort_flag) return false;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > kWaitNs) break;
   }
-  atomicExch(status, CSA_ERR_TIMEOUT);
+  atomicCAS(status, 0, CSA_ERR_TIMEOUT | (site << 8));
   *abort_flag = 1;
   return false;
 }
+#define tc_wait(bar, parity, status, abort_flag) tc_wait_site(bar, parity, status, abort_flag, __LINE__)
 
 __device__ __forceinline__ float redux_max(float v) {
   float r;
@@ -108,6 +158,25 @@ __device__ __forceinline__ float fast_ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
+// d = a * b + c and x += y on pairs of floats (packed f32x2 pipe ops).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fadd2(float& x0, float& x1, float y0, float y1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(y0), "f"(y1));
+}
+// Running-max sentinel for a column that has seen no valid row yet (finite, so
+// every softmax argument stays finite; masked rows are -inf and give 0).
+constexpr float kNoRowMax = -1e30f;
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -142,7 +211,7 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
 }
 
 template <int NB>
-__global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const TcArgs args) {
+__global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const TcArgs args, const __grid_constant__ TcMaps maps) {
   using C = TcCfg<NB>;
   constexpr int N = C::N;
   extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
@@ -159,7 +228,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       mbar_init(&sm.kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.q_full[s], 32 * C::kProdWarps);
+      mbar_init(&sm.q_full[s], 1);
       mbar_init(&sm.q_empty[s], 1 + 128 * C::kGroups);
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.s_free[s], 128 * C::kGroups);
@@ -171,6 +240,11 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     sm.abort_flag = 0;
     fence_mbar_init();
   }
+  for (int h = threadIdx.x; h < 128; h += blockDim.x)
+    sm.sink_l2[h] = (args.sink != nullptr && h < args.H) ? args.sink[h] * 1.4426950408889634f : -INFINITY;
+  for (int o = threadIdx.x * 16; o < C::kOnesBytes; o += blockDim.x * 16)
+    *reinterpret_cast<uint4*>(sm.ones + o) = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  fence_proxy_async();
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem, C::kTmemCols);
     tmem_relinquish();
@@ -182,7 +256,12 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
 
   if (warp >= kProd0 && warp < kMmaWarp) {
     // ===================================================================== producer
-    const int pt = threadIdx.x - 32 * kProd0;   // 0..63
+    const int pw = warp - kProd0;              // producer warp pw: tile rows [RW pw, RW pw + RW)
+    constexpr int RW = kTcTile / C::kProdWarps;
+    constexpr int NI = RW / 32;
+    const uint64_t map_q = reinterpret_cast<uint64_t>(&maps.q);
+    const uint64_t map_kv = reinterpret_cast<uint64_t>(&maps.kv);
+    const uint64_t map_raw = reinterpret_cast<uint64_t>(&maps.raw);
     int it = 0, kvc = 0;
     for (int u = blockIdx.x; u < args.n_units; u += gridDim.x, ++it) {
       if (*abort_flag) break;
@@ -195,6 +274,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       const int plast = p0 + ntok - 1;
       int n_c;
       const int32_t* irow = args.idx + (static_cast<size_t>(b) * args.T_chunk + r0) * args.k;
+      // top-k indices of this lane's rows (RW pw + 32 q + lane) of every entry
+      // tile, loaded up front
+      int ir[kTcMaxIdxTiles][NI];
       if (args.sparse) {
         // indices are ascending with -1 padding at the end: binary-search the count
         int lo = 0, hi = args.k;
@@ -203,53 +285,98 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           if (irow[mid] >= 0) lo = mid + 1; else hi = mid;
         }
         n_c = lo;
+#pragma unroll
+        for (int i = 0; i < kTcMaxIdxTiles; ++i)
+#pragma unroll
+          for (int q = 0; q < NI; ++q) {
+            const int L = i * kTcTile + RW * pw + 32 * q + lane;
+            ir[i][q] = L < n_c ? irow[L] : 0;
+          }
       } else {
         n_c = min(args.S, (plast + 1) / args.m);
       }
+      const int n_cp = (n_c + 3) & ~3;
       int jlo = 0, n_w = 0;
       if (args.W > 0) {
         jlo = max(0, p0 - args.W + 1);
         n_w = plast - jlo + 1;
       }
-      const int n_rows = n_c + n_w;
+      const int n_rows = n_cp + n_w;
       const int nt = max(1, (n_rows + kTcTile - 1) / kTcTile);
-      const int n_all = args.G > 1 ? min(n_c, (p0 + 1) / args.m) : n_rows;
-      if (pt == 0) sm.info[slot] = TcUnit{b, r0, ntok, n_c, n_w, jlo, p0, nt, n_all};
-      // ---- Q: N rows (token-major, head-minor), 16 chunks of 16 B each
-      {
-        const uint32_t qs = smem_u32(sm.q[slot]);
-        const size_t qrow0 = (static_cast<size_t>(b) * args.Tq + args.row0 + r0) * args.H;
-        for (int i = pt; i < N * 16; i += 32 * C::kProdWarps) {
-          const int row = i >> 4, ch = i & 15;
-          const bool ok = row < ntok * args.H;
-          const __nv_bfloat16* src = args.q + (ok ? (qrow0 + row) * kTcDim + ch * 8 : 0);
-          cp_async16(qs + sw128_off(row, ch, N), src, ok ? 16u : 0u);
+      const int n_all = args.G > 1 ? min(n_c, (p0 + 1) / args.m) : (n_c == n_cp ? n_rows : n_c);
+      if (pw == 0 && lane == 0) {
+        sm.info[slot] = TcUnit{b, r0, ntok, n_c, n_w, jlo, p0, nt, n_all, n_cp};
+        // ---- Q: per token one box of H rows (token-major, head-minor) per
+        // 64-column half; only the unit's ntok tokens, so no box leaves q
+        const int qrow0 = (b * args.Tq + args.row0 + r0) * args.H;
+        mbar_arrive_expect_tx(&sm.q_full[slot], ntok * args.H * kTcDim * 2);
+        for (int g = 0; g < ntok; ++g) {
+          const uint32_t qd = smem_u32(sm.q[slot]) + g * args.H * 128;
+          tma_load_2d(qd, map_q, 0, qrow0 + g * args.H, &sm.q_full[slot]);
+          tma_load_2d(qd + N * 128, map_q, 64, qrow0 + g * args.H, &sm.q_full[slot]);
         }
-        cp_async_mbar_arrive(&sm.q_full[slot]);
       }
       // ---- KV tiles
       for (int i = 0; i < nt; ++i, ++kvc) {
         const int stage = kvc % C::kStages;
         const int use = kvc / C::kStages;
         if (use >= 1 && !tc_wait(&sm.kv_empty[stage], (use - 1) & 1, args.status, abort_flag)) break;
+        if (pw == 0 && lane == 0) CSA_TR(it, i, 0);
+        const int L0 = i * kTcTile;
         const uint32_t ks = smem_u32(sm.kv[stage]);
-#pragma unroll
-        for (int rr2 = 0; rr2 < kTcTile / (32 * C::kProdWarps); ++rr2) {
-          const int rr = pt + rr2 * 32 * C::kProdWarps;
-          const int L = i * kTcTile + rr;
-          const __nv_bfloat16* src = nullptr;
-          if (L < n_c) {
-            const int s = args.sparse ? irow[L] : L;
-            src = args.kv_c + (static_cast<size_t>(b) * args.kv_bstride + s) * kTcDim;
-          } else if (L < n_rows) {
-            const int j = jlo + (L - n_c);
-            src = args.kv_raw + (static_cast<size_t>(b) * args.raw_cap + (j % args.raw_cap)) * kTcDim;
+        // contiguous tiles (every row valid and consecutive in one tensor) take two TMA boxes
+        const bool dense_entries = !args.sparse && L0 + kTcTile <= n_c;
+        const int wj = jlo + (L0 - n_cp);
+        const bool window_tile = L0 >= n_cp && L0 + kTcTile <= n_rows && (wj % args.raw_cap) + kTcTile <= args.raw_cap;
+        if (dense_entries || window_tile) {
+          if (pw == 0 && lane == 0) {
+            const uint64_t map = dense_entries ? map_kv : map_raw;
+            const int y = dense_entries ? b * args.kv_bstride + L0 : b * args.raw_cap + (wj % args.raw_cap);
+            mbar_arrive_expect_tx(&sm.kv_full[stage], kTcTile * kTcDim * 2);
+            tma_load_2d(ks, map, 0, y, &sm.kv_full[stage]);
+            tma_load_2d(ks + kTcTile * 128, map, 64, y, &sm.kv_full[stage]);
+          } else {
+            mbar_arrive(&sm.kv_full[stage]);
           }
+        } else {
+          // gather: each instruction moves two 256-byte rows (lanes 0-15 / 16-31)
+          int tr[NI];
 #pragma unroll
-          for (int ch = 0; ch < 16; ++ch)
-            cp_async16(ks + sw128_off(rr, ch, kTcTile), src ? src + ch * 8 : args.kv_c, src ? 16u : 0u);
+          for (int q = 0; q < NI; ++q) tr[q] = 0;
+#pragma unroll
+          for (int ii = 0; ii < kTcMaxIdxTiles; ++ii)
+            if (ii == i) {
+#pragma unroll
+              for (int q = 0; q < NI; ++q) tr[q] = ir[ii][q];
+            }
+          const int half = lane >> 4, c = lane & 15;
+#pragma unroll 8
+          for (int j = 0; j < RW / 2; ++j) {
+            const int rl = 2 * j + half;                   // row within this warp's RW rows
+            int s_g = 0;
+#pragma unroll
+            for (int q = 0; q < NI; ++q) {
+              const int v = __shfl_sync(0xffffffffu, tr[q], rl & 31);
+              if ((rl >> 5) == q) s_g = v;
+            }
+            const int rr = RW * pw + rl;                   // tile row
+            const int L = L0 + rr;
+            const __nv_bfloat16* src = args.kv_c;
+            uint32_t bytes = 0;
+            if (L < n_c) {
+              const int s = args.sparse ? s_g : L;
+              src = args.kv_c + (static_cast<size_t>(b) * args.kv_bstride + s) * kTcDim + c * 8;
+              bytes = 16;
+            } else if (L >= n_cp && L < n_rows) {
+              const int jj = jlo + (L - n_cp);
+              src = args.kv_raw + (static_cast<size_t>(b) * args.raw_cap + (jj % args.raw_cap)) * kTcDim + c * 8;
+              bytes = 16;
+            }
+            cp_async16(ks + sw128_off(rr, c, kTcTile), src, bytes);
+          }
+          cp_async_mbar_arrive(&sm.kv_full[stage]);
         }
-        cp_async_mbar_arrive(&sm.kv_full[stage]);
+        if (pw == 0 && lane == 0) CSA_TR(it, i, 1);
       }
     }
     cp_async_wait<0>();
@@ -258,6 +385,8 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, N, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, N, 1, 1);
+      constexpr uint32_t idesc_sum = idesc_bf16(128, N, 0, 1);
+      const uint32_t ones_base = smem_u32(sm.ones);
       int it = 0, kvc = 0, gt = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < args.n_units && ok; u += gridDim.x, ++it) {
@@ -274,6 +403,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           if (suse >= 1 && !tc_wait(&sm.s_free[sb], (suse - 1) & 1, args.status, abort_flag)) return false;
           fence_proxy_async();
           tc_fence_after();
+          CSA_TR(it, i, 2);
           const uint32_t kb = smem_u32(sm.kv[stage]);
 #pragma unroll
           for (int j = 0; j < kTcDim / 16; ++j)
@@ -294,6 +424,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           }
           fence_proxy_async();
           tc_fence_after();
+          CSA_TR(it, i, 3);
           const int stage = (kvc + i) % C::kStages;
           const uint32_t kb = smem_u32(sm.kv[stage]);
           const uint32_t pbase = smem_u32(sm.p[pb]);
@@ -301,6 +432,12 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           for (int j = 0; j < kTcTile / 16; ++j)
             mma_bf16(tmem + 2 * N + ob * N, desc_mnmajor(kb, kTcTile * 128, j), desc_mnmajor(pbase, kTcTile * 128, j),
                      idesc_pv, (i > 0 || j > 0) ? 1u : 0u);
+          if constexpr (C::kSumMma) {
+#pragma unroll
+            for (int j = 0; j < kTcTile / 16; ++j)
+              mma_bf16(tmem + 4 * N + ob * N, desc_kmajor(ones_base, 0, j), desc_mnmajor(pbase, kTcTile * 128, j),
+                       idesc_sum, (i > 0 || j > 0) ? 1u : 0u);
+          }
           tc_commit(&sm.kv_empty[stage]);
           tc_commit(&sm.p_empty[pb]);
         }
@@ -312,7 +449,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < C::kSoftWarps) {
     // ===================================================================== softmax
     const int wg = warp >> 2, wq = warp & 3;    // warpgroup wg owns columns [32 wg, 32 wg + 32)
     const int row = wq * 32 + lane;             // TMEM lane: KV tile row / O^T dim row
@@ -320,23 +457,31 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     const int col0 = 32 * wg;
     const float sl2 = args.scale_log2;
+    constexpr bool kSumMma = C::kSumMma;
     int it = 0, gt = 0;
     for (int u = blockIdx.x; u < args.n_units; u += gridDim.x, ++it) {
       const int slot = it & 1;
       if (!tc_wait(&sm.q_full[slot], (it >> 1) & 1, args.status, abort_flag)) break;
       const TcUnit inf = sm.info[slot];
-      const int n_rows = inf.n_c + inf.n_w;
+      const int n_rows = inf.n_cp + inf.n_w;
       const int ob = it & 1, ouse = it >> 1;
-      float lpart[32];
+      // running column maxima in registers (same in every thread of the
+      // warpgroup); per-thread row-sum partials unless the MMA keeps the sums
+      float mreg[32];
+      float lpart[kSumMma ? 1 : 32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) lpart[c] = 0.f;
-      if (row < 32) sm.mcol[wg][row] = -INFINITY;
+      for (int c = 0; c < 32; ++c) mreg[c] = kNoRowMax;
+#pragma unroll
+      for (int c = 0; c < (kSumMma ? 1 : 32); ++c) lpart[c] = 0.f;
+      if (row < 32) sm.mcol[wg][row] = kNoRowMax;
+      bool allset = false;   // every column of this warpgroup has a running max
       named_bar_sync(bar_id, 128);
       bool ok = true;
       for (int i = 0; i < inf.nt; ++i, ++gt) {
         const int sb = gt & 1;
         if (!tc_wait(&sm.s_full[sb], (gt >> 1) & 1, args.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        if (threadIdx.x == 0) CSA_TR(it, i, 4);
         float s[32];
         {
           uint32_t v[32];
@@ -347,11 +492,12 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         }
         tc_fence_before();
         mbar_arrive(&sm.s_free[sb]);
+        if (threadIdx.x == 0 && i < 8) CSA_TR(it, 8 + i, 0);
         // ---- masks (only tiles that reach past the rows every token sees):
         // padding rows, and for multi-token units per-token visibility
         if ((i + 1) * kTcTile > inf.n_all) {
           const int L = i * kTcTile + row;
-          if (L >= n_rows) {
+          if (L >= n_rows || (L >= inf.n_c && L < inf.n_cp)) {
 #pragma unroll
             for (int c = 0; c < 32; ++c) s[c] = -INFINITY;
           } else if (args.G > 1) {
@@ -362,7 +508,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
               if (L < inf.n_c) {
                 vis = args.m * (L + 1) - 1 <= p;
               } else {
-                const int j = inf.jlo + (L - inf.n_c);
+                const int j = inf.jlo + (L - inf.n_cp);
                 vis = j <= p && j > p - args.W;
               }
               if (vis && g < inf.ntok) vmask |= 1u << g;
@@ -372,67 +518,106 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
               if (!((vmask >> ((col0 + c) >> args.hshift)) & 1u)) s[c] = -INFINITY;
           }
         }
-        // ---- column maxima: warp redux, then 4-warp exchange
+        // ---- d = s * scale_log2 - m in place (m = running column max, kept in
+        // registers).  The exact column max of d (warp redux + 4-warp exchange)
+        // is taken when some d exceeds 2^8 or a column sees its first valid row
+        // (always on a unit's first tile); otherwise one barrier-OR suffices.
+        float dmax = -INFINITY;
+        bool newrow = false;
+        if (allset) {
 #pragma unroll
-        for (int c4 = 0; c4 < 32; c4 += 4) {
-          const float a0 = redux_max(s[c4]), a1 = redux_max(s[c4 + 1]);
-          const float a2 = redux_max(s[c4 + 2]), a3 = redux_max(s[c4 + 3]);
-          if (lane == 0) *reinterpret_cast<float4*>(&sm.xch[wg][wq][c4]) = make_float4(a0, a1, a2, a3);
-        }
-        named_bar_sync(bar_id, 128);
-        bool need = false;
-        if (row < 32) {
-          const int c = row;
-          const float tmax = fmaxf(fmaxf(sm.xch[wg][0][c], sm.xch[wg][1][c]), fmaxf(sm.xch[wg][2][c], sm.xch[wg][3][c]));
-          const float tm = tmax * sl2;
-          const float mo = sm.mcol[wg][c];
-          float mn = mo, a = 1.f;
-          if (tm > mo + 8.0f) {
-            mn = tm;
-            a = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
-            need = (i > 0) && (mo != -INFINITY);
+          for (int c = 0; c < 32; c += 2) {
+            ffma2(s[c], s[c + 1], s[c], s[c + 1], sl2, sl2, -mreg[c], -mreg[c + 1]);
+            dmax = fmaxf(dmax, fmaxf(s[c], s[c + 1]));
           }
-          sm.mcol[wg][c] = mn;
-          sm.alpha[wg][c] = a;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const bool sen = mreg[c] == kNoRowMax;
+            s[c] = fmaf(s[c], sl2, sen ? 0.f : -mreg[c]);
+            if (sen) newrow |= s[c] > -INFINITY;
+            else dmax = fmaxf(dmax, s[c]);
+          }
         }
-        const bool rescale = bar_red_or(bar_id, 128, need);
-        if (rescale) {
-          // rare: the running max rose by more than 2^8; PV(i-1) must be complete
-          const int gp = gt - 1;
-          if (!tc_wait(&sm.p_empty[gp & 1], (gp >> 1) & 1, args.status, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t oaddr = tmem + lane_addr + 2 * N + ob * N + col0;
+        const bool full_max = bar_red_or(bar_id, 128, dmax > 8.0f || newrow);
+        if (threadIdx.x == 0 && i < 8) CSA_TR(it, 8 + i, 1);
+        if (full_max) {
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t v[16];
-            tmem_ld16(oaddr + 16 * h2, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float a = sm.alpha[wg][16 * h2 + c];
-              v[c] = __float_as_uint(__uint_as_float(v[c]) * a);
-              lpart[16 * h2 + c] *= a;
+          for (int c4 = 0; c4 < 32; c4 += 4) {
+            const float a0 = redux_max(s[c4]), a1 = redux_max(s[c4 + 1]);
+            const float a2 = redux_max(s[c4 + 2]), a3 = redux_max(s[c4 + 3]);
+            if (lane == 0) *reinterpret_cast<float4*>(&sm.xch[wg][wq][c4]) = make_float4(a0, a1, a2, a3);
+          }
+          named_bar_sync(bar_id, 128);
+          if (threadIdx.x == 0) CSA_TR(it, i, 6);
+          bool need = false, unset = false;
+          if (row < 32) {
+            const int c = row;
+            const float x = fmaxf(fmaxf(sm.xch[wg][0][c], sm.xch[wg][1][c]), fmaxf(sm.xch[wg][2][c], sm.xch[wg][3][c]));
+            const float mo = sm.mcol[wg][c];
+            float mn = mo, a = 1.f, delta = 0.f;
+            if (mo == kNoRowMax) {
+              if (x > -INFINITY) { mn = x; delta = x; }   // first valid rows: d was s * scale
+            } else if (x > 8.0f) {
+              mn = mo + x; delta = x; a = exp2f(-x); need = i > 0;
             }
-            tmem_st16(oaddr + 16 * h2, v);
+            sm.mcol[wg][c] = mn;
+            sm.alpha[wg][c] = a;
+            sm.dlt[wg][c] = delta;
+            unset = mn == kNoRowMax;
           }
-          tmem_st_wait();
-          tc_fence_before();
+          const bool rescale = bar_red_or(bar_id, 128, need);
+          const bool any_unset = bar_red_or(bar_id, 128, unset);
+          if (threadIdx.x == 0) CSA_TR(it, i, 7);
+          allset = !any_unset;
+#pragma unroll
+          for (int c4 = 0; c4 < 32; c4 += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(&sm.mcol[wg][c4]);
+            const float4 d4 = *reinterpret_cast<const float4*>(&sm.dlt[wg][c4]);
+            mreg[c4] = m4.x; mreg[c4 + 1] = m4.y; mreg[c4 + 2] = m4.z; mreg[c4 + 3] = m4.w;
+            s[c4] -= d4.x; s[c4 + 1] -= d4.y; s[c4 + 2] -= d4.z; s[c4 + 3] -= d4.w;
+          }
+          if (rescale) {
+            // rare: the running max rose by more than 2^8; PV(i-1) must be complete
+            const int gp = gt - 1;
+            if (!tc_wait(&sm.p_empty[gp & 1], (gp >> 1) & 1, args.status, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int buf = 0; buf < (kSumMma ? 2 : 1); ++buf) {
+              // O^T, and with the row-sum MMA also L^T, share the column scaling
+              const uint32_t oaddr = tmem + lane_addr + (2 + 2 * buf) * N + ob * N + col0;
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t v[16];
+                tmem_ld16(oaddr + 16 * h2, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                  v[c] = __float_as_uint(__uint_as_float(v[c]) * sm.alpha[wg][16 * h2 + c]);
+                tmem_st16(oaddr + 16 * h2, v);
+              }
+            }
+            if constexpr (!kSumMma) {
+#pragma unroll
+              for (int c = 0; c < (kSumMma ? 1 : 32); ++c) lpart[c] *= sm.alpha[wg][c];
+            }
+            tmem_st_wait();
+            tc_fence_before();
+          }
         }
-        // ---- P^T = 2^(s * scale_log2 - m), row sums, bf16 into shared memory
+        // ---- P^T = 2^d (bf16) into shared memory (+ per-thread row sums)
         const int pb = gt & 1, puse = gt >> 1;
         if (puse >= 1 && !tc_wait(&sm.p_empty[pb], (puse - 1) & 1, args.status, abort_flag)) { ok = false; break; }
+        if (threadIdx.x == 0 && i < 8) CSA_TR(it, 8 + i, 2);
         const uint32_t prow = smem_u32(sm.p[pb]) + (wg >> 1) * (kTcTile * 128) + row * 128;
 #pragma unroll
         for (int c8 = 0; c8 < 32; c8 += 8) {
-          const float4 m0 = *reinterpret_cast<const float4*>(&sm.mcol[wg][c8]);
-          const float4 m1 = *reinterpret_cast<const float4*>(&sm.mcol[wg][c8 + 4]);
-          const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
           float pv[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float me = mm[e] == -INFINITY ? 0.f : mm[e];
-            pv[e] = fast_ex2(fmaf(s[c8 + e], sl2, -me));
-            lpart[c8 + e] += pv[e];
+          for (int e = 0; e < 8; e += 2) {
+            pv[e] = fast_ex2(s[c8 + e]);
+            pv[e + 1] = fast_ex2(s[c8 + e + 1]);
+            if constexpr (!kSumMma) fadd2(lpart[(c8 + e) % (kSumMma ? 1 : 32)], lpart[(c8 + e + 1) % (kSumMma ? 1 : 32)], pv[e], pv[e + 1]);
           }
           const uint32_t w0 = pack_bf16(pv[0], pv[1]), w1 = pack_bf16(pv[2], pv[3]);
           const uint32_t w2 = pack_bf16(pv[4], pv[5]), w3 = pack_bf16(pv[6], pv[7]);
@@ -441,68 +626,87 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1), "r"(w2), "r"(w3)
                        : "memory");
         }
+        if (threadIdx.x == 0 && i < 8) CSA_TR(it, 8 + i, 3);
         fence_proxy_async();
         mbar_arrive(&sm.p_full[pb]);
+        if (threadIdx.x == 0) CSA_TR(it, i, 5);
       }
       if (!ok) break;
-      // ---- unit epilogue: column sums of lpart over the 128 rows (butterfly:
-      // lane l ends with column l's warp total), then the 4-warp total
+      if (threadIdx.x == 0) CSA_TR(it, 14, 0);
+      // ---- unit epilogue: per-column row sums l (TMEM L^T, or the 128 rows'
+      // partials: butterfly so lane l ends with column l's warp total, then the
+      // 4-warp total), output scale 2^(m-M) / (l 2^(m-M) + 2^(sigma-M)) with
+      // M = max(m, sigma), and lse (natural log, sink excluded)
+      if constexpr (!kSumMma) {
 #pragma unroll
-      for (int st = 16; st >= 1; st >>= 1) {
-        const bool up = (lane & st) != 0;
+        for (int st = 16; st >= 1; st >>= 1) {
+          const bool up = (lane & st) != 0;
 #pragma unroll
-        for (int e = 0; e < st; ++e) {
-          const float send = up ? lpart[e] : lpart[e + st];
-          const float keep = up ? lpart[e + st] : lpart[e];
-          lpart[e] = keep + __shfl_xor_sync(0xffffffffu, send, st);
+          for (int e = 0; e < st; ++e) {
+            const float send = up ? lpart[e % (kSumMma ? 1 : 32)] : lpart[(e + st) % (kSumMma ? 1 : 32)];
+            const float keep = up ? lpart[(e + st) % (kSumMma ? 1 : 32)] : lpart[e % (kSumMma ? 1 : 32)];
+            lpart[e % (kSumMma ? 1 : 32)] = keep + __shfl_xor_sync(0xffffffffu, send, st);
+          }
         }
+        sm.xch[wg][wq][lane] = lpart[0];
+        named_bar_sync(bar_id, 128);
       }
-      sm.xch[wg][wq][lane] = lpart[0];
-      named_bar_sync(bar_id, 128);
-      if (row < 32) {
-        const int c = row;
-        sm.alpha[wg][c] = (sm.xch[wg][0][c] + sm.xch[wg][1][c]) + (sm.xch[wg][2][c] + sm.xch[wg][3][c]);
-      }
-      named_bar_sync(bar_id, 128);
       if (!tc_wait(&sm.o_full[ob], ouse & 1, args.status, abort_flag)) break;
       tc_fence_after();
+      if (threadIdx.x == 0) CSA_TR(it, 15, 6);
+      if (wq == 0) {
+        // warp 0 of the warpgroup: lane c handles column col0 + c
+        const int c = lane;
+        float l;
+        if constexpr (kSumMma) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_addr + 4 * N + ob * N + col0, v);   // every lane holds all column sums
+          tmem_ld_wait();
+          l = 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (e == c) l = __uint_as_float(v[e]);
+        } else {
+          l = (sm.xch[wg][0][c] + sm.xch[wg][1][c]) + (sm.xch[wg][2][c] + sm.xch[wg][3][c]);
+        }
+        const float mcl = sm.mcol[wg][c];
+        const int col = col0 + c;
+        const int h = col & (args.H - 1);
+        float scale = 0.f, lse_v = -INFINITY;
+        if (mcl > 0.5f * kNoRowMax) {
+          const float sg = sm.sink_l2[h];
+          const float mx = fmaxf(mcl, sg);
+          const float f = exp2f(mcl - mx);
+          const float den = fmaf(l, f, exp2f(sg - mx));
+          scale = den > 0.f ? __fdiv_rn(f, den) : 0.f;
+          if (l > 0.f) lse_v = (mcl + log2f(l)) * 0.6931471805599453f;
+        }
+        sm.alpha[wg][c] = scale;
+        const int g = col >> args.hshift;
+        if (args.lse != nullptr && g < inf.ntok)
+          args.lse[(static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + g) * args.H + h] = lse_v;
+      }
+      named_bar_sync(bar_id, 128);
+      if (threadIdx.x == 0) CSA_TR(it, 14, 1);
       {
         const uint32_t oaddr = tmem + lane_addr + 2 * N + ob * N + col0;
         const int d = row;
         uint32_t v[32];
         tmem_ld32(oaddr, v);
         tmem_ld_wait();
+        if (threadIdx.x == 0) CSA_TR(it, 14, 2);
+        __nv_bfloat16* obase = args.out + (static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0) * args.H * kTcDim + d;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int col = col0 + c;
-          const int g = col >> args.hshift, h = col & (args.H - 1);
-          if (g >= inf.ntok) continue;
-          const float mcl = sm.mcol[wg][c];
-          const float l = sm.alpha[wg][c];
-          float res = 0.f;
-          if (mcl != -INFINITY) {
-            const float sg = args.sink ? args.sink[h] * 1.4426950408889634f : -INFINITY;
-            const float mx = fmaxf(mcl, sg);
-            const float f = exp2f(mcl - mx);
-            const float den = fmaf(l, f, exp2f(sg - mx));
-            res = den > 0.f ? __fdiv_rn(__uint_as_float(v[c]) * f, den) : 0.f;
-          }
-          const size_t orow = (static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + g) * args.H + h;
-          args.out[orow * kTcDim + d] = __float2bfloat16_rn(res);
+          if ((col >> args.hshift) >= inf.ntok) continue;
+          obase[static_cast<size_t>(col) * kTcDim] = __float2bfloat16_rn(__uint_as_float(v[c]) * sm.alpha[wg][c]);
         }
       }
+      if (threadIdx.x == 0) CSA_TR(it, 14, 3);
       tc_fence_before();
       mbar_arrive(&sm.o_empty[ob]);
-      if (args.lse != nullptr && row < 32) {
-        const int col = col0 + row;
-        const int g = col >> args.hshift, h = col & (args.H - 1);
-        if (g < inf.ntok) {
-          const float mcl = sm.mcol[wg][row];
-          const float l = sm.alpha[wg][row];
-          const float v = (mcl == -INFINITY || !(l > 0.f)) ? -INFINITY : (mcl + log2f(l)) * 0.6931471805599453f;
-          args.lse[(static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + g) * args.H + h] = v;
-        }
-      }
+      if (threadIdx.x == 0) CSA_TR(it, 15, 7);
       named_bar_sync(bar_id, 128);      // mcol / alpha reused by the next unit
       mbar_arrive(&sm.q_empty[slot]);
     }
@@ -515,8 +719,35 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
   }
 }
 
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 map over [rows, 128] with 128-byte swizzle and a 64 x box_rows box.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kTcDim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kTcDim) * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
 template <int NB>
-int launch_attn_tc_nb(const TcArgs& a, cudaStream_t st) {
+int launch_attn_tc_nb(const TcArgs& a, const TcMaps& maps, cudaStream_t st) {
   const size_t smem = sizeof(TcSmem<NB>) + 1024;
   static bool attr_set = false;
   if (!attr_set) {
@@ -529,7 +760,7 @@ int launch_attn_tc_nb(const TcArgs& a, cudaStream_t st) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = a.n_units < sms ? a.n_units : sms;
-  attn_tc_kernel<NB><<<grid, TcCfg<NB>::kThreads, smem, st>>>(a);
+  attn_tc_kernel<NB><<<grid, TcCfg<NB>::kThreads, smem, st>>>(a, maps);
   return check_launch();
 }
 
@@ -568,7 +799,20 @@ int launch_attn_tc(const void* q, const void* kv_c, const int32_t* idx, const vo
   CSA_REQUIRE(nu < (1ll << 31), CSA_ERR_UNSUPPORTED);
   a.n_units = static_cast<int>(nu);
   if (a.n_units == 0) return CSA_OK;
-  return N == 64 ? launch_attn_tc_nb<1>(a, st) : launch_attn_tc_nb<2>(a, st);
+  if (sparse) CSA_REQUIRE(k <= kTcMaxIdxTiles * kTcTile, CSA_ERR_UNSUPPORTED);
+  const long long q_rows = static_cast<long long>(B) * Tq * H;
+  const long long kv_rows = static_cast<long long>(B) * kv_bstride;
+  const long long raw_rows = static_cast<long long>(B) * a.raw_cap;
+  CSA_REQUIRE(q_rows < (1ll << 31) && kv_rows < (1ll << 31) - 1 && raw_rows < (1ll << 31) - 1, CSA_ERR_UNSUPPORTED);
+  a.kv_rows = static_cast<int>(kv_rows);
+  a.raw_rows = static_cast<int>(raw_rows);
+  TcMaps maps;
+  if (!make_map(&maps.q, q, static_cast<uint64_t>(q_rows), static_cast<uint32_t>(H)) ||
+      !make_map(&maps.kv, kv_c, static_cast<uint64_t>(kv_rows), kTcTile) ||
+      !make_map(&maps.raw, kv_raw ? kv_raw : kv_c, static_cast<uint64_t>(kv_raw ? raw_rows : kv_rows), kTcTile))
+    return CSA_ERR_CUDA;
+  if (!kv_raw) a.raw_rows = a.kv_rows;
+  return N == 64 ? launch_attn_tc_nb<1>(a, maps, st) : launch_attn_tc_nb<2>(a, maps, st);
 }
 
 }  // namespace csa

@@ -4,56 +4,59 @@
 //
 // Radix select on order-preserving integer keys: a float's bit pattern is
 // mapped so that unsigned integer order equals float order (+0 and -0 map to
-// the same key).  8-bit digits are resolved from the top; each pass builds a
-// 256-bin histogram of the candidates that still match the chosen prefix, and
-// the bin holding the k-th largest key fixes the next digit.  After the last
-// pass the threshold key K is exact: every key > K is selected, and the
-// (k - #greater) keys == K with the smallest indices.  The final pass is an
-// in-order compaction (block-wide prefix sums), so indices come out ascending
-// and the result is bit-exact and independent of scheduling.
+// the same key); BF16 rows use 16-bit keys, FP32 rows 32-bit keys.  8-bit
+// digits are resolved from the top: a 256-bin histogram of the candidates that
+// still match the chosen prefix (per-warp shared-memory histograms), one block
+// scan over the bins, and the bin holding the k-th largest key fixes the next
+// digit.  After the last digit the threshold key K is exact: every key > K is
+// selected, plus the (k - #greater) keys == K with the smallest indices.
 //
-// One CTA per query row; the visible prefix of the row is staged in shared
-// memory when it fits, otherwise every pass re-reads it from L2.
+// The output is an in-order compaction: each warp owns a contiguous segment of
+// the row and walks it 32 keys at a time with ballots, so indices come out
+// ascending, shared-memory reads are conflict-free, and only the warps'
+// totals cross a barrier.  Bit-exact and independent of scheduling.
+//
+// One CTA (256 threads) per query row; the visible prefix of the row is staged
+// in shared memory when it fits, otherwise every pass re-reads it from L2.
 #include "common.cuh"
 
 namespace csa {
 
-constexpr int kTopkThreads = 512;
+constexpr int kTopkThreads = 256;
 constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr size_t kTopkSmemMax = 160 * 1024;
 
-__device__ __forceinline__ uint32_t key_of(float x) {
-  uint32_t u = __float_as_uint(x);
-  if (u == 0x80000000u) u = 0u;                       // -0 == +0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ uint32_t key_of(__nv_bfloat16 x) {
-  uint32_t u = __bfloat16_as_ushort(x);
-  if (u == 0x8000u) u = 0u;
-  return (u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u);
-}
+template <typename T> struct KeyOf;
+template <> struct KeyOf<float> {
+  using K = uint32_t;
+  static constexpr int bits = 32;
+  static __device__ __forceinline__ K get(float x) {
+    uint32_t u = __float_as_uint(x);
+    if (u == 0x80000000u) u = 0u;                       // -0 == +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  }
+};
+template <> struct KeyOf<__nv_bfloat16> {
+  using K = uint16_t;
+  static constexpr int bits = 16;
+  static __device__ __forceinline__ K get(__nv_bfloat16 x) {
+    uint32_t u = __bfloat16_as_ushort(x);
+    if (u == 0x8000u) u = 0u;
+    return static_cast<K>((u & 0x8000u) ? (~u & 0xFFFFu) : (u | 0x8000u));
+  }
+};
 
-template <typename T> struct KeyBits;
-template <> struct KeyBits<float> { static constexpr int bits = 32; };
-template <> struct KeyBits<__nv_bfloat16> { static constexpr int bits = 16; };
-
-// Block-wide exclusive scan of one int per thread (in thread order); also
-// returns the block total.  Uses `scratch` (kTopkWarps + 1 ints).
-__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
+// Inclusive scan of one int per thread across the CTA (thread order).
+__device__ __forceinline__ int block_incl_scan(int v, int* wsum) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int inc = warp_incl_scan(v);
-  if (lane == 31) scratch[warp] = inc;
+  if (lane == 31) wsum[warp] = inc;
   __syncthreads();
-  if (warp == 0) {
-    int w = lane < kTopkWarps ? scratch[lane] : 0;
-    const int wi = warp_incl_scan(w);
-    if (lane < kTopkWarps) scratch[lane] = wi - w;
-    if (lane == kTopkWarps - 1) scratch[kTopkWarps] = wi;
-  }
+  int before = 0;
+#pragma unroll
+  for (int w = 0; w < kTopkWarps; ++w) before += (w < warp) ? wsum[w] : 0;
   __syncthreads();
-  const int res = scratch[warp] + inc - v;
-  *total = scratch[kTopkWarps];
-  __syncthreads();
-  return res;
+  return before + inc;
 }
 
 template <typename T, bool kSmem>
@@ -61,11 +64,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const T* __restr
                                                                int ld, int k, int m, int row0,
                                                                const int32_t* __restrict__ q_pos0,
                                                                int32_t* __restrict__ idx) {
+  using KO = KeyOf<T>;
+  using K = typename KO::K;
   extern __shared__ __align__(16) uint8_t dsm[];
   __shared__ int hist[kTopkWarps][256];
-  __shared__ int scratch[kTopkWarps + 2];
-  __shared__ uint32_t sel_digit;
-  __shared__ int sel_above;
+  __shared__ int wsum[kTopkWarps];
+  __shared__ int wcnt[kTopkWarps][2];
+  __shared__ int sel_digit, sel_above;
 
   const int row = blockIdx.x;
   const int bi = row / T_chunk;
@@ -76,87 +81,128 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const T* __restr
   if (nv < 0) nv = 0;
   const int n = static_cast<int>(nv);
   int32_t* out = idx + static_cast<size_t>(row) * k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (n <= k) {
-    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = i < n ? i : -1;
+    for (int i = tid; i < k; i += kTopkThreads) out[i] = i < n ? i : -1;
     return;
   }
   const T* srow = score + static_cast<size_t>(row) * ld;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(dsm);
+  K* keys = reinterpret_cast<K*>(dsm);
   if (kSmem) {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = key_of(srow[i]);
+    // 16-byte loads (several in flight per thread), keys stored 16 bytes at a time
+    constexpr int V = 16 / sizeof(T);
+    int done = 0;
+    if ((reinterpret_cast<uintptr_t>(srow) & 15) == 0) {
+      const int nvec = n / V;
+#pragma unroll 4
+      for (int j = tid; j < nvec; j += kTopkThreads) {
+        const uint4 u = reinterpret_cast<const uint4*>(srow)[j];
+        const T* e = reinterpret_cast<const T*>(&u);
+        K kk[V];
+#pragma unroll
+        for (int q = 0; q < V; ++q) kk[q] = KO::get(e[q]);
+        if constexpr (sizeof(K) * V == 16) {
+          *reinterpret_cast<uint4*>(keys + static_cast<size_t>(j) * V) = *reinterpret_cast<const uint4*>(kk);
+        } else {
+#pragma unroll
+          for (int q = 0; q < V; ++q) keys[static_cast<size_t>(j) * V + q] = kk[q];
+        }
+      }
+      done = nvec * V;
+    }
+    for (int i = done + tid; i < n; i += kTopkThreads) keys[i] = KO::get(srow[i]);
+    __syncthreads();
   }
-  auto key_at = [&](int i) -> uint32_t { return kSmem ? keys[i] : key_of(srow[i]); };
+  auto key_at = [&](int i) -> K { return kSmem ? keys[i] : KO::get(srow[i]); };
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t prefix = 0, pmask = 0;
   int krem = k;
-  constexpr int kBits = KeyBits<T>::bits;
 #pragma unroll 1
-  for (int shift = kBits - 8; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < kTopkWarps * 256; i += blockDim.x) (&hist[0][0])[i] = 0;
+  for (int shift = KO::bits - 8; shift >= 0; shift -= 8) {
+#pragma unroll
+    for (int w = 0; w < kTopkWarps; ++w) hist[w][tid] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t key = key_at(i);
-      const bool cand = (key & pmask) == prefix;
+    for (int base = 0; base < n; base += kTopkThreads) {
+      const int i = base + tid;
+      const uint32_t key = i < n ? static_cast<uint32_t>(key_at(i)) : 0u;
+      const bool cand = i < n && (key & pmask) == prefix;
       const uint32_t dig = (key >> shift) & 0xFFu;
-      // warp-aggregated increment of the per-warp histogram
-      const unsigned act = __ballot_sync(__activemask(), cand);
-      if (cand) {
-        const unsigned peers = __match_any_sync(act, dig);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[warp][dig], __popc(peers));
-      }
+      if (cand) atomicAdd(&hist[warp][dig], 1);
     }
     __syncthreads();
-    if (warp == 0) {
-      // lane l owns digits 255-8l .. 248-8l (descending); count per digit
-      int cnt[8];
-      int tot = 0;
+    // thread t owns digit 255 - t: the inclusive scan in thread order counts
+    // the candidates with a digit >= 255 - t
+    const int d = 255 - tid;
+    int c = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int d = 255 - (8 * lane + j);
-        int c = 0;
-        for (int w = 0; w < kTopkWarps; ++w) c += hist[w][d];
-        cnt[j] = c;
-        tot += c;
-      }
-      const int incl = warp_incl_scan(tot);
-      int before = incl - tot;         // # candidates with a larger digit than this lane's first
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (before < krem && krem <= before + cnt[j]) {
-          sel_digit = static_cast<uint32_t>(255 - (8 * lane + j));
-          sel_above = before;
-        }
-        before += cnt[j];
-      }
+    for (int w = 0; w < kTopkWarps; ++w) c += hist[w][d];
+    const int incl = block_incl_scan(c, wsum);
+    const int above = incl - c;
+    if (above < krem && krem <= incl) {
+      sel_digit = d;
+      sel_above = above;
     }
     __syncthreads();
-    prefix |= sel_digit << shift;
+    prefix |= static_cast<uint32_t>(sel_digit) << shift;
     pmask |= 0xFFu << shift;
     krem -= sel_above;
-    __syncthreads();
   }
-  // threshold key = prefix; take all keys > prefix, and the first `krem` keys == prefix.
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int i0 = min(n, static_cast<int>(threadIdx.x) * per);
-  const int i1 = min(n, i0 + per);
+  // threshold key = prefix; take every key > prefix and the first `krem` keys == prefix.
+  const int seg = (n + kTopkWarps * 32 - 1) / (kTopkWarps * 32) * 32;
+  const int s0 = warp * seg, s1 = min(n, s0 + seg);
   int n_gt = 0, n_eq = 0;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t key = key_at(i);
-    n_gt += key > prefix;
-    n_eq += key == prefix;
+  for (int b0 = s0; b0 < s1; b0 += 32) {
+    const int i = b0 + lane;
+    const uint32_t key = i < s1 ? static_cast<uint32_t>(key_at(i)) : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, i < s1 && key > prefix));
+    n_eq += __popc(__ballot_sync(0xffffffffu, i < s1 && key == prefix));
   }
-  int tot;
-  const int eq_before = block_excl_scan(n_eq, scratch, &tot);
-  const int eq_take = max(0, min(n_eq, krem - eq_before));
-  const int pos0 = block_excl_scan(n_gt + eq_take, scratch, &tot);
-  int o = pos0, eq_seen = 0;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t key = key_at(i);
-    bool take = key > prefix;
-    if (key == prefix) { take = eq_seen < eq_take; ++eq_seen; }
-    if (take) out[o++] = i;
+  if (lane == 0) {
+    wcnt[warp][0] = n_gt;
+    wcnt[warp][1] = n_eq;
   }
+  __syncthreads();
+  int out_pos = 0, eq_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    const int take_eq = max(0, min(wcnt[w][1], krem - eq_before));
+    out_pos += wcnt[w][0] + take_eq;
+    eq_before += wcnt[w][1];
+  }
+  const unsigned below = (1u << lane) - 1u;
+  for (int b0 = s0; b0 < s1; b0 += 32) {
+    const int i = b0 + lane;
+    const uint32_t key = i < s1 ? static_cast<uint32_t>(key_at(i)) : 0u;
+    const bool gt = i < s1 && key > prefix;
+    const bool eq = i < s1 && key == prefix;
+    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_before + __popc(eqm & below) < krem);
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[out_pos + __popc(tm & below)] = i;
+    out_pos += __popc(tm);
+    eq_before += __popc(eqm);
+  }
+}
+
+template <typename T>
+int launch_topk(const T* score, int B, int T_chunk, int S, int ld, int k, int m, int row0, const int32_t* q_pos0,
+                int32_t* idx, cudaStream_t st) {
+  const long long rows = static_cast<long long>(B) * T_chunk;
+  using K = typename KeyOf<T>::K;
+  const size_t keys_bytes = static_cast<size_t>(S) * sizeof(K);
+  const unsigned grid = static_cast<unsigned>(rows);
+  if (keys_bytes <= kTopkSmemMax) {
+    static int attr = -1;
+    if (attr < static_cast<int>(keys_bytes)) {
+      cudaError_t e = cudaFuncSetAttribute(topk_row_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kTopkSmemMax));
+      if (e != cudaSuccess) return set_cuda_error(e);
+      attr = static_cast<int>(kTopkSmemMax);
+    }
+    topk_row_kernel<T, true><<<grid, kTopkThreads, keys_bytes, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, idx);
+  } else {
+    topk_row_kernel<T, false><<<grid, kTopkThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, idx);
+  }
+  return check_launch();
 }
 
 }  // namespace csa
@@ -182,31 +228,10 @@ int topk_select(const void* score, int score_dtype, int B, int T_chunk, int S, i
   if (rows == 0) return CSA_OK;
   CSA_REQUIRE(rows < (1ll << 31), CSA_ERR_UNSUPPORTED);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t keys_bytes = static_cast<size_t>(S) * 4;
-  const bool smem = keys_bytes <= 160 * 1024;
-  const unsigned grid = static_cast<unsigned>(rows);
-  if (score_dtype == CSA_F32) {
-    if (smem) {
-      cudaFuncSetAttribute(topk_row_kernel<float, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(keys_bytes));
-      topk_row_kernel<float, true><<<grid, kTopkThreads, keys_bytes, st>>>(
-          static_cast<const float*>(score), T_chunk, S, score_ld, k, m, row0, q_pos0, idx);
-    } else {
-      topk_row_kernel<float, false><<<grid, kTopkThreads, 0, st>>>(static_cast<const float*>(score), T_chunk, S,
-                                                                    score_ld, k, m, row0, q_pos0, idx);
-    }
-  } else {
-    if (smem) {
-      cudaFuncSetAttribute(topk_row_kernel<__nv_bfloat16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(keys_bytes));
-      topk_row_kernel<__nv_bfloat16, true><<<grid, kTopkThreads, keys_bytes, st>>>(
-          static_cast<const __nv_bfloat16*>(score), T_chunk, S, score_ld, k, m, row0, q_pos0, idx);
-    } else {
-      topk_row_kernel<__nv_bfloat16, false><<<grid, kTopkThreads, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(score), T_chunk, S, score_ld, k, m, row0, q_pos0, idx);
-    }
-  }
-  return check_launch();
+  if (score_dtype == CSA_F32)
+    return launch_topk(static_cast<const float*>(score), B, T_chunk, S, score_ld, k, m, row0, q_pos0, idx, st);
+  return launch_topk(static_cast<const __nv_bfloat16*>(score), B, T_chunk, S, score_ld, k, m, row0, q_pos0, idx,
+                     st);
 }
 
 }  // extern "C"

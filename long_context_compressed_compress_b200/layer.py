@@ -23,6 +23,18 @@ from . import ops
 _DT = {"bf16": torch.bfloat16, "f32": torch.float32}
 
 
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def _no_timer(name):
+    return _Null()
+
+
 class CsaPrefill:
     """Buffers + call sequence of one CSA prefill layer.  ``chunk`` bounds the
     query rows scored at once (the score buffer is [B, chunk, S])."""
@@ -47,23 +59,31 @@ class CsaPrefill:
         self.q_pos0 = torch.zeros((c.B,), dtype=torch.int32, device=device)
         self.launches = 3 + 3 * ((c.T + self.chunk - 1) // self.chunk)
 
-    def run(self, x, keep_idx=None):
+    def run(self, x, keep_idx=None, timer=None):
         """x: dict of device tensors (input generator order).  If ``keep_idx`` is a
-        tensor [B, T, k] the selected indices of every chunk are copied into it."""
+        tensor [B, T, k] the selected indices of every chunk are copied into it.
+        ``timer(name)`` may return a context manager wrapped around each call."""
         c = self.cfg
-        ops.csa_compress(x["a"], x["b"], x["z"], c.m, out=self.kv_c)
-        ops.csa_compress(x["a_I"], x["b_I"], x["z_I"], c.m, out_fp4=self.k_fp4, out_sf=self.k_sf,
-                         gscale=self.g, out_dtype=x["a_I"].dtype)
-        ops.nvfp4_quantize(x["q_I"], self.q_fp4, self.q_sf, self.g)
+        t = timer or _no_timer
+        with t("csa_compress"):
+            ops.csa_compress(x["a"], x["b"], x["z"], c.m, out=self.kv_c)
+        with t("csa_compress_indexer_keys"):
+            ops.csa_compress(x["a_I"], x["b_I"], x["z_I"], c.m, out_fp4=self.k_fp4, out_sf=self.k_sf,
+                             gscale=self.g, out_dtype=x["a_I"].dtype)
+        with t("nvfp4_quantize"):
+            ops.nvfp4_quantize(x["q_I"], self.q_fp4, self.q_sf, self.g)
         for r0 in range(0, c.T, self.chunk):
             tc = min(self.chunk, c.T - r0)
             sc = self.score.view(-1)[: c.B * tc * c.S].view(c.B, tc, c.S)
             ix = self.idx.view(-1)[: c.B * tc * c.k].view(c.B, tc, c.k)
-            ops.indexer_score(self.q_fp4, self.q_sf, self.k_fp4, self.k_sf, x["w"], self.q_pos0, sc, c.S, c.m,
-                              row0=r0, T_chunk=tc, q_gscale=self.g, k_gscale=self.g)
-            ops.topk_select(sc, ix, c.S, c.m, self.q_pos0, row0=r0)
-            ops.sparse_attn_fwd(x["q"], self.kv_c, ix, x["kv_raw"], x["sink"], c.tau, c.W, self.q_pos0,
-                                self.out, self.lse, row0=r0, T_chunk=tc)
+            with t("indexer_score"):
+                ops.indexer_score(self.q_fp4, self.q_sf, self.k_fp4, self.k_sf, x["w"], self.q_pos0, sc, c.S, c.m,
+                                  row0=r0, T_chunk=tc, q_gscale=self.g, k_gscale=self.g)
+            with t("topk_select"):
+                ops.topk_select(sc, ix, c.S, c.m, self.q_pos0, row0=r0)
+            with t("sparse_attn_fwd"):
+                ops.sparse_attn_fwd(x["q"], self.kv_c, ix, x["kv_raw"], x["sink"], c.tau, c.W, self.q_pos0,
+                                    self.out, self.lse, row0=r0, T_chunk=tc)
             if keep_idx is not None:
                 keep_idx[:, r0:r0 + tc].copy_(ix)
         return self.out
@@ -82,9 +102,12 @@ class HcaPrefill:
         self.q_pos0 = torch.zeros((c.B,), dtype=torch.int32, device=device)
         self.launches = 2
 
-    def run(self, x):
+    def run(self, x, timer=None):
         c = self.cfg
-        ops.hca_compress(x["a"], x["z"], c.m, self.kv_c)
-        ops.hca_dense_attn_fwd(x["q"], self.kv_c, x["kv_raw"], x["sink"], c.tau, c.W, self.q_pos0, self.out, c.m,
-                               lse=self.lse)
+        t = timer or _no_timer
+        with t("hca_compress"):
+            ops.hca_compress(x["a"], x["z"], c.m, self.kv_c)
+        with t("hca_dense_attn_fwd"):
+            ops.hca_dense_attn_fwd(x["q"], self.kv_c, x["kv_raw"], x["sink"], c.tau, c.W, self.q_pos0, self.out,
+                                   c.m, lse=self.lse)
         return self.out
