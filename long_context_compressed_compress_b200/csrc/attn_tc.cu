@@ -22,8 +22,8 @@
 //     zero-filled by out-of-range coordinates) so a group never mixes sources.
 //   MMA warp (1): issues QK(i+1) before PV(i) so the tensor core works on the
 //     next tile while the softmax runs.
-//   softmax warpgroups (N/64, 4 warps each): thread = TMEM lane = KV row of S^T
-//     and dim row of O^T; a warpgroup owns 64 columns.  Column maxima are warp
+//   softmax warpgroups (4 warps each): thread = TMEM lane = KV row of S^T
+//     and dim row of O^T; a warpgroup owns 16 (N = 64) or 32 (N = 128) columns.  Column maxima are warp
 //     redux.sync.max + a 4-warp exchange; running maxima are raised only when a
 //     tile exceeds them by 2^8 (then O^T and the row sums are rescaled), row
 //     sums stay per thread until the unit's end.  P^T goes to shared memory as
@@ -43,7 +43,7 @@ __device__ unsigned long long* g_csa_trace;
   do {                                                                                           \
     if (blockIdx.x == 0 && g_csa_trace != nullptr && (unit) < 64 && (tile) < 16) {               \
       unsigned long long t_;                                                                     \
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                     \
+      asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_));                                         \
       g_csa_trace[((unit) * 16 + (tile)) * 8 + (ev)] = t_;                                        \
     }                                                                                            \
   } while (0)
@@ -59,11 +59,12 @@ namespace csa {
 constexpr int kTcTile = 128;   // KV rows per tile
 constexpr int kTcDim = 128;    // head dim
 
-// NB = number of 64-column blocks of N; each softmax warpgroup owns 32 columns.
+// NB = number of 64-column blocks of N; each softmax warpgroup owns kCW columns.
 template <int NB>
 struct TcCfg {
   static constexpr int N = 64 * NB;                       // MMA N (token, head) columns
-  static constexpr int kGroups = N / 32;                  // softmax warpgroups
+  static constexpr int kCW = NB == 1 ? 16 : 32;            // columns per softmax warpgroup
+  static constexpr int kGroups = N / kCW;                  // softmax warpgroups
   static constexpr int kSoftWarps = 4 * kGroups;
   static constexpr int kProdWarps = NB == 1 ? 4 : 2;   // gather issue rate scales with warps
   static constexpr int kThreads = 32 * (kSoftWarps + kProdWarps + 1);
@@ -101,10 +102,10 @@ struct __align__(1024) TcSmem {
   uint8_t ones[C::kOnesBytes];   // bf16 1.0 (A operand of the row-sum MMA)
   uint64_t kv_full[C::kStages], kv_empty[C::kStages];
   uint64_t q_full[2], q_empty[2], s_full[2], s_free[2], p_full[2], p_empty[2], o_full[2], o_empty[2];
-  float xch[2 * NB][4][32];
-  float mcol[2 * NB][32];
-  float alpha[2 * NB][32];
-  float dlt[2 * NB][32];
+  float xch[C::kGroups][4][C::kCW];
+  float mcol[C::kGroups][C::kCW];
+  float alpha[C::kGroups][C::kCW];
+  float dlt[C::kGroups][C::kCW];
   float sink_l2[128];      // sink logits in log2 units (-inf without a sink)
   TcUnit info[2];
   uint32_t tmem;
@@ -451,11 +452,12 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     __syncwarp();
   } else if (warp < C::kSoftWarps) {
     // ===================================================================== softmax
-    const int wg = warp >> 2, wq = warp & 3;    // warpgroup wg owns columns [32 wg, 32 wg + 32)
+    constexpr int CW = C::kCW;
+    const int wg = warp >> 2, wq = warp & 3;    // warpgroup wg owns columns [CW wg, CW wg + CW)
     const int row = wq * 32 + lane;             // TMEM lane: KV tile row / O^T dim row
     const int bar_id = 1 + wg;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-    const int col0 = 32 * wg;
+    const int col0 = CW * wg;
     const float sl2 = args.scale_log2;
     constexpr bool kSumMma = C::kSumMma;
     int it = 0, gt = 0;
@@ -467,13 +469,13 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       const int ob = it & 1, ouse = it >> 1;
       // running column maxima in registers (same in every thread of the
       // warpgroup); per-thread row-sum partials unless the MMA keeps the sums
-      float mreg[32];
-      float lpart[kSumMma ? 1 : 32];
+      float mreg[CW];
+      float lpart[kSumMma ? 1 : CW];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) mreg[c] = kNoRowMax;
+      for (int c = 0; c < CW; ++c) mreg[c] = kNoRowMax;
 #pragma unroll
-      for (int c = 0; c < (kSumMma ? 1 : 32); ++c) lpart[c] = 0.f;
-      if (row < 32) sm.mcol[wg][row] = kNoRowMax;
+      for (int c = 0; c < (kSumMma ? 1 : CW); ++c) lpart[c] = 0.f;
+      if (row < CW) sm.mcol[wg][row] = kNoRowMax;
       bool allset = false;   // every column of this warpgroup has a running max
       named_bar_sync(bar_id, 128);
       bool ok = true;
@@ -482,13 +484,14 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         if (!tc_wait(&sm.s_full[sb], (gt >> 1) & 1, args.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (threadIdx.x == 0) CSA_TR(it, i, 4);
-        float s[32];
+        float s[CW];
         {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_addr + sb * N + col0, v);
+          uint32_t v[CW];
+          tmem_ld16(tmem + lane_addr + sb * N + col0, v);
+          if constexpr (CW == 32) tmem_ld16(tmem + lane_addr + sb * N + col0 + 16, v + 16);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(v[c]);
+          for (int c = 0; c < CW; ++c) s[c] = __uint_as_float(v[c]);
         }
         tc_fence_before();
         mbar_arrive(&sm.s_free[sb]);
@@ -499,7 +502,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           const int L = i * kTcTile + row;
           if (L >= n_rows || (L >= inf.n_c && L < inf.n_cp)) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) s[c] = -INFINITY;
+            for (int c = 0; c < CW; ++c) s[c] = -INFINITY;
           } else if (args.G > 1) {
             uint32_t vmask = 0;
             for (int g = 0; g < args.G; ++g) {
@@ -514,7 +517,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
               if (vis && g < inf.ntok) vmask |= 1u << g;
             }
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
+            for (int c = 0; c < CW; ++c)
               if (!((vmask >> ((col0 + c) >> args.hshift)) & 1u)) s[c] = -INFINITY;
           }
         }
@@ -526,32 +529,55 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         bool newrow = false;
         if (allset) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
+          for (int c = 0; c < CW; c += 2) {
             ffma2(s[c], s[c + 1], s[c], s[c + 1], sl2, sl2, -mreg[c], -mreg[c + 1]);
             dmax = fmaxf(dmax, fmaxf(s[c], s[c + 1]));
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
+          for (int c = 0; c < CW; ++c) {
             const bool sen = mreg[c] == kNoRowMax;
             s[c] = fmaf(s[c], sl2, sen ? 0.f : -mreg[c]);
             if (sen) newrow |= s[c] > -INFINITY;
             else dmax = fmaxf(dmax, s[c]);
           }
         }
+        // ---- P^T = 2^d (bf16) into shared memory (+ per-thread row sums).
+        // P buffer gt & 1 was last read by PV(gt - 2), which the MMA issued before
+        // QK(gt); s_full(gt) completing implies it completed, so no wait here.
+        const int pb = gt & 1;
+        const uint32_t prow = smem_u32(sm.p[pb]) + (col0 >> 6) * (kTcTile * 128) + row * 128;
+        auto store_p = [&]() {
+#pragma unroll
+          for (int c8 = 0; c8 < CW; c8 += 8) {
+            float pv[8];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              pv[e] = fast_ex2(s[c8 + e]);
+              pv[e + 1] = fast_ex2(s[c8 + e + 1]);
+              if constexpr (!kSumMma)
+                fadd2(lpart[(c8 + e) % (kSumMma ? 1 : CW)], lpart[(c8 + e + 1) % (kSumMma ? 1 : CW)], pv[e], pv[e + 1]);
+            }
+            const uint32_t w0 = pack_bf16(pv[0], pv[1]), w1 = pack_bf16(pv[2], pv[3]);
+            const uint32_t w2 = pack_bf16(pv[4], pv[5]), w3 = pack_bf16(pv[6], pv[7]);
+            const int chunk = ((col0 & 63) >> 3) + (c8 >> 3);
+            const uint32_t addr = prow + ((chunk ^ (row & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1), "r"(w2), "r"(w3)
+                         : "memory");
+          }
+        };
         const bool full_max = bar_red_or(bar_id, 128, dmax > 8.0f || newrow);
         if (threadIdx.x == 0 && i < 8) CSA_TR(it, 8 + i, 1);
         if (full_max) {
 #pragma unroll
-          for (int c4 = 0; c4 < 32; c4 += 4) {
+          for (int c4 = 0; c4 < CW; c4 += 4) {
             const float a0 = redux_max(s[c4]), a1 = redux_max(s[c4 + 1]);
             const float a2 = redux_max(s[c4 + 2]), a3 = redux_max(s[c4 + 3]);
             if (lane == 0) *reinterpret_cast<float4*>(&sm.xch[wg][wq][c4]) = make_float4(a0, a1, a2, a3);
           }
           named_bar_sync(bar_id, 128);
           if (threadIdx.x == 0) CSA_TR(it, i, 6);
-          bool need = false, unset = false;
-          if (row < 32) {
+          if (row < CW) {
             const int c = row;
             const float x = fmaxf(fmaxf(sm.xch[wg][0][c], sm.xch[wg][1][c]), fmaxf(sm.xch[wg][2][c], sm.xch[wg][3][c]));
             const float mo = sm.mcol[wg][c];
@@ -559,24 +585,28 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
             if (mo == kNoRowMax) {
               if (x > -INFINITY) { mn = x; delta = x; }   // first valid rows: d was s * scale
             } else if (x > 8.0f) {
-              mn = mo + x; delta = x; a = exp2f(-x); need = i > 0;
+              mn = mo + x; delta = x; a = exp2f(-x);
             }
             sm.mcol[wg][c] = mn;
             sm.alpha[wg][c] = a;
             sm.dlt[wg][c] = delta;
-            unset = mn == kNoRowMax;
           }
-          const bool rescale = bar_red_or(bar_id, 128, need);
-          const bool any_unset = bar_red_or(bar_id, 128, unset);
+          named_bar_sync(bar_id, 128);
           if (threadIdx.x == 0) CSA_TR(it, i, 7);
-          allset = !any_unset;
+          // every thread reads the same arrays, so these decisions are uniform
+          bool rescale = false, any_unset = false;
 #pragma unroll
-          for (int c4 = 0; c4 < 32; c4 += 4) {
+          for (int c4 = 0; c4 < CW; c4 += 4) {
             const float4 m4 = *reinterpret_cast<const float4*>(&sm.mcol[wg][c4]);
             const float4 d4 = *reinterpret_cast<const float4*>(&sm.dlt[wg][c4]);
+            const float4 a4 = *reinterpret_cast<const float4*>(&sm.alpha[wg][c4]);
             mreg[c4] = m4.x; mreg[c4 + 1] = m4.y; mreg[c4 + 2] = m4.z; mreg[c4 + 3] = m4.w;
             s[c4] -= d4.x; s[c4 + 1] -= d4.y; s[c4 + 2] -= d4.z; s[c4 + 3] -= d4.w;
+            rescale |= (a4.x != 1.f) | (a4.y != 1.f) | (a4.z != 1.f) | (a4.w != 1.f);
+            any_unset |= (m4.x == kNoRowMax) | (m4.y == kNoRowMax) | (m4.z == kNoRowMax) | (m4.w == kNoRowMax);
           }
+          rescale = rescale && i > 0;
+          allset = !any_unset;
           if (rescale) {
             // rare: the running max rose by more than 2^8; PV(i-1) must be complete
             const int gp = gt - 1;
@@ -587,7 +617,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
               // O^T, and with the row-sum MMA also L^T, share the column scaling
               const uint32_t oaddr = tmem + lane_addr + (2 + 2 * buf) * N + ob * N + col0;
 #pragma unroll
-              for (int h2 = 0; h2 < 2; ++h2) {
+              for (int h2 = 0; h2 < CW / 16; ++h2) {
                 uint32_t v[16];
                 tmem_ld16(oaddr + 16 * h2, v);
                 tmem_ld_wait();
@@ -599,33 +629,13 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
             }
             if constexpr (!kSumMma) {
 #pragma unroll
-              for (int c = 0; c < (kSumMma ? 1 : 32); ++c) lpart[c] *= sm.alpha[wg][c];
+              for (int c = 0; c < (kSumMma ? 1 : CW); ++c) lpart[c] *= sm.alpha[wg][c];
             }
             tmem_st_wait();
             tc_fence_before();
           }
         }
-        // ---- P^T = 2^d (bf16) into shared memory (+ per-thread row sums)
-        const int pb = gt & 1, puse = gt >> 1;
-        if (puse >= 1 && !tc_wait(&sm.p_empty[pb], (puse - 1) & 1, args.status, abort_flag)) { ok = false; break; }
-        if (threadIdx.x == 0 && i < 8) CSA_TR(it, 8 + i, 2);
-        const uint32_t prow = smem_u32(sm.p[pb]) + (wg >> 1) * (kTcTile * 128) + row * 128;
-#pragma unroll
-        for (int c8 = 0; c8 < 32; c8 += 8) {
-          float pv[8];
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            pv[e] = fast_ex2(s[c8 + e]);
-            pv[e + 1] = fast_ex2(s[c8 + e + 1]);
-            if constexpr (!kSumMma) fadd2(lpart[(c8 + e) % (kSumMma ? 1 : 32)], lpart[(c8 + e + 1) % (kSumMma ? 1 : 32)], pv[e], pv[e + 1]);
-          }
-          const uint32_t w0 = pack_bf16(pv[0], pv[1]), w1 = pack_bf16(pv[2], pv[3]);
-          const uint32_t w2 = pack_bf16(pv[4], pv[5]), w3 = pack_bf16(pv[6], pv[7]);
-          const int chunk = (wg & 1) * 4 + (c8 >> 3);
-          const uint32_t addr = prow + ((chunk ^ (row & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1), "r"(w2), "r"(w3)
-                       : "memory");
-        }
+        store_p();
         if (threadIdx.x == 0 && i < 8) CSA_TR(it, 8 + i, 3);
         fence_proxy_async();
         mbar_arrive(&sm.p_full[pb]);
@@ -643,9 +653,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           const bool up = (lane & st) != 0;
 #pragma unroll
           for (int e = 0; e < st; ++e) {
-            const float send = up ? lpart[e % (kSumMma ? 1 : 32)] : lpart[(e + st) % (kSumMma ? 1 : 32)];
-            const float keep = up ? lpart[(e + st) % (kSumMma ? 1 : 32)] : lpart[e % (kSumMma ? 1 : 32)];
-            lpart[e % (kSumMma ? 1 : 32)] = keep + __shfl_xor_sync(0xffffffffu, send, st);
+            const float send = up ? lpart[e % (kSumMma ? 1 : CW)] : lpart[(e + st) % (kSumMma ? 1 : CW)];
+            const float keep = up ? lpart[(e + st) % (kSumMma ? 1 : CW)] : lpart[e % (kSumMma ? 1 : CW)];
+            lpart[e % (kSumMma ? 1 : CW)] = keep + __shfl_xor_sync(0xffffffffu, send, st);
           }
         }
         sm.xch[wg][wq][lane] = lpart[0];
@@ -655,21 +665,22 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       tc_fence_after();
       if (threadIdx.x == 0) CSA_TR(it, 15, 6);
       if (wq == 0) {
-        // warp 0 of the warpgroup: lane c handles column col0 + c
-        const int c = lane;
+        // warp 0 of the warpgroup: lane c < CW handles column col0 + c
+        const int c = lane % CW;
         float l;
         if constexpr (kSumMma) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_addr + 4 * N + ob * N + col0, v);   // every lane holds all column sums
+          uint32_t v[CW];
+          tmem_ld16(tmem + lane_addr + 4 * N + ob * N + col0, v);   // every lane holds all column sums
+          if constexpr (CW == 32) tmem_ld16(tmem + lane_addr + 4 * N + ob * N + col0 + 16, v + 16);
           tmem_ld_wait();
           l = 0.f;
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
+          for (int e = 0; e < CW; ++e)
             if (e == c) l = __uint_as_float(v[e]);
         } else {
           l = (sm.xch[wg][0][c] + sm.xch[wg][1][c]) + (sm.xch[wg][2][c] + sm.xch[wg][3][c]);
         }
-        const float mcl = sm.mcol[wg][c];
+        const float mcl = mreg[0] * 0.f + sm.mcol[wg][c];
         const int col = col0 + c;
         const int h = col & (args.H - 1);
         float scale = 0.f, lse_v = -INFINITY;
@@ -681,9 +692,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           scale = den > 0.f ? __fdiv_rn(f, den) : 0.f;
           if (l > 0.f) lse_v = (mcl + log2f(l)) * 0.6931471805599453f;
         }
-        sm.alpha[wg][c] = scale;
+        if (lane < CW) sm.alpha[wg][c] = scale;
         const int g = col >> args.hshift;
-        if (args.lse != nullptr && g < inf.ntok)
+        if (args.lse != nullptr && lane < CW && g < inf.ntok)
           args.lse[(static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + g) * args.H + h] = lse_v;
       }
       named_bar_sync(bar_id, 128);
@@ -691,13 +702,14 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       {
         const uint32_t oaddr = tmem + lane_addr + 2 * N + ob * N + col0;
         const int d = row;
-        uint32_t v[32];
-        tmem_ld32(oaddr, v);
+        uint32_t v[CW];
+        tmem_ld16(oaddr, v);
+        if constexpr (CW == 32) tmem_ld16(oaddr + 16, v + 16);
         tmem_ld_wait();
         if (threadIdx.x == 0) CSA_TR(it, 14, 2);
         __nv_bfloat16* obase = args.out + (static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0) * args.H * kTcDim + d;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < CW; ++c) {
           const int col = col0 + c;
           if ((col >> args.hshift) >= inf.ntok) continue;
           obase[static_cast<size_t>(col) * kTcDim] = __float2bfloat16_rn(__uint_as_float(v[c]) * sm.alpha[wg][c]);

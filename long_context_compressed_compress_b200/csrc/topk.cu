@@ -16,13 +16,14 @@
 // ascending, shared-memory reads are conflict-free, and only the warps'
 // totals cross a barrier.  Bit-exact and independent of scheduling.
 //
-// One CTA (256 threads) per query row; the visible prefix of the row is staged
+// One CTA (128 threads) per query row; the visible prefix of the row is staged
 // in shared memory when it fits, otherwise every pass re-reads it from L2.
 #include "common.cuh"
 
 namespace csa {
 
-constexpr int kTopkThreads = 256;
+constexpr int kTopkThreads = 128;
+constexpr int kTopkDpt = 256 / kTopkThreads;   // histogram digits per thread in the scan
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr size_t kTopkSmemMax = 160 * 1024;
 
@@ -120,7 +121,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const T* __restr
 #pragma unroll 1
   for (int shift = KO::bits - 8; shift >= 0; shift -= 8) {
 #pragma unroll
-    for (int w = 0; w < kTopkWarps; ++w) hist[w][tid] = 0;
+    for (int w = 0; w < kTopkWarps; ++w)
+#pragma unroll
+      for (int q = 0; q < kTopkDpt; ++q) hist[w][tid + q * kTopkThreads] = 0;
     __syncthreads();
     for (int base = 0; base < n; base += kTopkThreads) {
       const int i = base + tid;
@@ -130,17 +133,26 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const T* __restr
       if (cand) atomicAdd(&hist[warp][dig], 1);
     }
     __syncthreads();
-    // thread t owns digit 255 - t: the inclusive scan in thread order counts
-    // the candidates with a digit >= 255 - t
-    const int d = 255 - tid;
-    int c = 0;
+    // thread t owns digits 255 - kTopkDpt t - q (descending): the inclusive scan
+    // in thread order counts the candidates with a larger-or-equal digit
+    int cq[kTopkDpt], csum = 0;
 #pragma unroll
-    for (int w = 0; w < kTopkWarps; ++w) c += hist[w][d];
-    const int incl = block_incl_scan(c, wsum);
-    const int above = incl - c;
-    if (above < krem && krem <= incl) {
-      sel_digit = d;
-      sel_above = above;
+    for (int q = 0; q < kTopkDpt; ++q) {
+      const int d = 255 - kTopkDpt * tid - q;
+      int c = 0;
+#pragma unroll
+      for (int w = 0; w < kTopkWarps; ++w) c += hist[w][d];
+      cq[q] = c;
+      csum += c;
+    }
+    int above = block_incl_scan(csum, wsum) - csum;
+#pragma unroll
+    for (int q = 0; q < kTopkDpt; ++q) {
+      if (above < krem && krem <= above + cq[q]) {
+        sel_digit = 255 - kTopkDpt * tid - q;
+        sel_above = above;
+      }
+      above += cq[q];
     }
     __syncthreads();
     prefix |= static_cast<uint32_t>(sel_digit) << shift;
