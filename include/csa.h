@@ -21,8 +21,9 @@
  *    packed E2M1 bytes (element 2i in the low nibble, 2i+1 in the high nibble)
  *    plus one E4M3 scale byte per 16 elements plus one fp32 global scale g > 0.
  *  - Positions: q_pos0[b] (device, int32) is the absolute position of query row
- *    0 of sequence b (0 for a prefill, the cache length for decode); query row r
- *    of a call sits at position p = q_pos0[b] + r.
+ *    0 of sequence b (0 for a prefill, the cache length for decode).  Calls that
+ *    take a row chunk [row0, row0 + T_chunk) place chunk row r at position
+ *    p = q_pos0[b] + row0 + r; the others place query row r at q_pos0[b] + r.
  *  - Visibility: compressed entry s is visible at position p iff
  *    m*(s+1) - 1 <= p (only completed blocks are visible).
  *  - Raw window: raw token j is visible at p iff p - W < j <= p and j >= 0; it
