@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=0,
                     help="profiling case: override the layer's token count (not a bench line)")
+    ap.add_argument("--workload", default="csa_prefill_32k", choices=["csa_prefill_32k", "csa_decode_32x1m"],
+                    help="csa_prefill_32k (the default line) or csa_decode_32x1m (decode steps/s)")
     return ap.parse_args()
 
 
@@ -258,6 +260,9 @@ def main():
     cfg = configs.CSA_PREFILL
     if args.T:
         cfg = configs.scaled(cfg, T=args.T)
+    if args.workload == "csa_decode_32x1m":
+        main_decode(args, rank, world, local)
+        return
     if args.impl == "reference":
         run_reference(args, cfg, rank)
         return
@@ -418,6 +423,182 @@ def main():
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_rows)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def decode_cpu_baseline(cfg, n_seq=2):
+    """The oracle's decode step on ``n_seq`` sequences of the same cache recipe
+    (state converted to float64 beforehand, not timed), extrapolated to B."""
+    import numpy as np
+    import oracle
+    from long_context_compressed_compress_b200 import inputs
+    import torch
+    st = inputs.decode_state(cfg)
+    seqs = list(range(n_seq))
+    f = lambda t: t.to(torch.float64).numpy()
+    o = {"kv_c": f(st["kv_c"][seqs, :cfg.S0]), "khat": oracle.nvfp4_quantize(f(st["k_I_src"][seqs, :cfg.S0]))["xhat"],
+         "ring": f(st["ring"][seqs]).copy()}
+    slot0 = ((cfg.T0 // cfg.m - 1) % 2) * cfg.m
+    for n in ("a", "b", "z", "a_I", "b_I", "z_I"):
+        src = f(st["carry_" + n][seqs])
+        buf = np.zeros((n_seq, 2 * cfg.m, src.shape[-1]))
+        buf[:, slot0:slot0 + cfg.m] = src
+        o["carry_" + n] = buf
+    x = {k: f(v[seqs]) for k, v in inputs.decode_step_inputs(cfg, 0).items()}
+    x["sink"] = f(st["sink"])
+    t0 = time.perf_counter()
+    oracle.csa_decode_step(o, x, cfg.T0, cfg.m, cfg.k, cfg.W, cfg.tau, cfg.dtype)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = 1
+    return {"value": 1.0 / (dt * cfg.B / n_seq), "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"one decode step for {n_seq} of the {cfg.B} sequences ({dt:.1f} s), "
+                      f"extrapolated to all {cfg.B}"}
+
+
+def main_decode(args, rank, world, local):
+    """CSA decode at 1M context: B = 32 sequences x 1,048,576 cached tokens
+    (262,144 entries), H = 128, k = 1024; one step = one new token for every
+    sequence, replayed from a CUDA graph.  value = steps/s of the whole job."""
+    import dataclasses
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import build, configs
+    build.build()
+    from long_context_compressed_compress_b200 import inputs, layer
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if args.impl == "reference":
+        if rank == 0:
+            cfg = configs.CSA_DECODE
+            cb = decode_cpu_baseline(cfg)
+            print(json.dumps({"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "steps/s",
+                              "n_gpus": args.gpus, "steps": 1, "warmup": 0, "higher_is_better": True,
+                              "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                              "config": {"workload": "csa_decode_32x1m"}, "cpu_baseline": cb,
+                              "e2e": {"value": cb["value"], "unit": "steps/s", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    n_kern = 8
+    total = args.warmup + args.steps + 2 * (args.e2e_steps + 2) + n_kern + 8
+    cfg = dataclasses.replace(configs.CSA_DECODE, steps=total)
+    peaks = load_peaks()
+    st = inputs.decode_state(cfg, device="cuda")
+    lay = layer.CsaDecode(cfg, st, cfg.T0)
+    stream = torch.cuda.current_stream()
+    x = inputs.decode_step_inputs(cfg, 0, device="cuda")
+    # per-kernel breakdown: eager steps with events around each call
+    ev = {}
+
+    @contextlib.contextmanager
+    def timer(name):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        yield
+        e1.record(stream)
+        ev.setdefault(name, []).append((e0, e1))
+
+    lay.step(x)
+    torch.cuda.synchronize()
+    for _ in range(n_kern):
+        lay.step(x, timer=timer)
+    torch.cuda.synchronize()
+    kern = {k: sum(a.elapsed_time(b) for a, b in v) / n_kern for k, v in ev.items()}
+    lay.capture(x)
+    for _ in range(args.warmup):
+        lay.replay()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(local))
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(args.steps):
+        lay.replay()
+    s1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    ms = s0.elapsed_time(s1)
+    if world > 1:
+        ms = max_over_ranks(ms, dev)
+    ms_step = ms / args.steps
+    # end to end: pinned host inputs copied in, the graph, the output read back
+    host = {k: v.cpu().pin_memory() for k, v in x.items()}
+    out_host = torch.empty(lay.out.shape, dtype=lay.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            lay.x[k].copy_(v, non_blocking=True)
+        lay.replay()
+        out_host.copy_(lay.out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / max(1, args.e2e_steps)
+    if world > 1:
+        e2e_ms = max_over_ranks(e2e_ms, dev)
+    # roofline of the dominant kernel (the indexer: reads every visible NVFP4 key)
+    B, DI, HI = cfg.B, cfg.DI, cfg.HI
+    n_vis = (cfg.T0 + 1) // cfg.m
+    idx_bytes = B * (n_vis * (DI // 2 + DI // 16) + n_vis * 2 + HI * (DI // 2 + DI // 16 + 4))
+    topk_bytes = B * (n_vis * 2 + cfg.k * 4)
+    attn_bytes = B * (cfg.H * cfg.D * 2 * 2 + (cfg.k + cfg.W) * cfg.D * 2 + cfg.k * 4)
+    rates = {"indexer_score": idx_bytes, "topk_select": topk_bytes, "sparse_attn_fwd": attn_bytes}
+    kernels = {}
+    for name, t in kern.items():
+        amount = rates.get(name)
+        rate = amount / (t * 1e-3) / 1e9 if amount and t > 0 else None
+        kernels[name] = {"ms": round(t, 5), "achieved": rate and round(rate, 1), "unit": "GB/s" if rate else "",
+                         "frac": rate and round(rate / peaks["hbm_gbs"], 4)}
+    it = kern["indexer_score"]
+    achieved = idx_bytes / (it * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": world / (ms_step * 1e-3), "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic cache drawn on the device (N(0,1) entries and indexer keys, seeded)",
+        "config": {"workload": "csa_decode_32x1m", "B": B, "T0": cfg.T0, "S0": cfg.S0, "H": cfg.H, "D": cfg.D,
+                   "HI": HI, "DI": DI, "k": cfg.k, "W": cfg.W, "graph": True,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (302 MB of NVFP4 keys and 2.1 GB of KV per step's cache)"},
+        "e2e": {"value": job_throughput(world, 1, e2e_ms), "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": lay.launches * args.steps,
+        "roofline": {"bound": "hbm", "kernel": "indexer_score", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peaks['source']} hbm_gbs", "algorithmic_bytes_per_launch": idx_bytes},
+        "kernels": kernels, "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = decode_cpu_baseline(configs.CSA_DECODE)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    lay.graph = None
     if world > 1:
         dist.destroy_process_group()
 

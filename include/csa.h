@@ -91,7 +91,8 @@ int csa_device_status(int* status_out);
  * [B, 2m, D] holding raw token j at slot j % (2m); with p = ring_pos[b], if
  * (p+1) % m == 0 the entry i = (p+1)/m - 1 is written at entry index i of the
  * outputs (whose batch stride is out_bstride entries), else nothing is written
- * for that sequence.
+ * for that sequence.  An entry index i >= out_bstride (a full cache) is not
+ * written.
  *
  * Outputs (either may be NULL, not both): out [B, out_bstride, D] in out_dtype;
  * NVFP4 out_fp4 [B, out_bstride, D/2] + out_sf [B, out_bstride, D/16] with
@@ -154,9 +155,15 @@ int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_gscale,
  *   score [B, T_chunk, score_ld] (CSA_F32 / CSA_BF16), visible prefix of row r
  *   has n_r = min(S, (q_pos0[b] + row0 + r + 1) / m) entries
  *   idx int32 [B, T_chunk, k]
- * Radix select on order-preserving integer keys; bit-exact.  workspace may be
- * NULL when topk_workspace_size() returns 0 for the shape; otherwise it must
- * hold that many bytes of device memory.  Scores must not be NaN.
+ * Radix select on order-preserving integer keys; bit-exact.  Scores must not
+ * be NaN.
+ * Workspace: topk_workspace_size() gives the bytes a shape can use (0 when it
+ * needs none).  It is non-zero for few (B*T_chunk <= 512) long (S >= 16384)
+ * rows, where BF16 rows are split across several CTAs that meet through the
+ * workspace (4-byte aligned device memory owned by the caller; its contents
+ * on entry do not matter, the call clears what it uses).  With workspace NULL
+ * or smaller than that, the call falls back to one CTA per row (same result,
+ * slower).  Calls that share a workspace must be ordered on one stream.
  */
 int topk_select(const void* score, int score_dtype, int B, int T_chunk, int S,
                 int score_ld, int k, int m, int row0, const int32_t* q_pos0,

@@ -68,8 +68,10 @@ __global__ void __launch_bounds__(256) csa_compress_kernel(
   } else {
     bi = static_cast<int>(g2 / G);
     const int p = ring_pos[bi];
-    active = valid && ((p + 1) % m == 0);
     const int i = (p + 1) / m - 1;
+    // an entry is emitted when block i completes; entries past the cache's
+    // capacity (out_bstride rows) are dropped rather than written out of bounds
+    active = valid && ((p + 1) % m == 0) && i >= 0 && i < out_bstride;
     cur0 = (i & 1) * m;
     pred0 = ((i + 1) & 1) * m;
     has_pred = i > 0;

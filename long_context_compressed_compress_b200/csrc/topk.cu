@@ -195,6 +195,254 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const T* __restr
   }
 }
 
+// ---------------------------------------------------------------------------
+// Multi-CTA select for a few long BF16 rows (decode: 32 rows of 262144 scores).
+// A row is cut into chunks of kMcChunk keys, one CTA per (row, chunk), and the
+// radix select runs as four launches that meet through a caller workspace:
+//   K1  11-bit histogram of the high key bits      -> ws hist1[row][2048]
+//   K2  threshold bin b1 (every CTA scans hist1),
+//       5-bit histogram of the keys in bin b1       -> ws hist2[row][32]
+//   K3  exact threshold key K and the count krem of keys == K to take;
+//       per-chunk counts of keys > K and == K       -> ws cnt[row][chunk][2]
+//   K4  in-order compaction: the chunk's output offset is the sum over earlier
+//       chunks, then per-warp segments with ballots, as in the one-CTA kernel.
+// The histograms are cleared by a memset at the start of every call.  The
+// union of per-chunk results is the exact row result with the same tie rule.
+// ---------------------------------------------------------------------------
+constexpr int kMcThreads = 256;
+constexpr int kMcWarps = kMcThreads / 32;
+constexpr int kMcChunk = 8192;
+constexpr int kMcHist1 = 2048;
+constexpr int kMcHist2 = 32;
+constexpr int kMcRowsMax = 512;     // more rows than this use one CTA per row
+constexpr int kMcMinS = 16384;      // shorter rows use one CTA per row
+
+struct McLayout {
+  int C;            // chunks per row
+  size_t row_ints;  // ints per row
+  // per row: hist1[2048] hist2[32] state[4] cnt[C][2]
+  static constexpr int kHist2 = kMcHist1, kState = kMcHist1 + kMcHist2, kCnt = kMcHist1 + kMcHist2 + 4;
+  __host__ __device__ McLayout(int S) : C((S + kMcChunk - 1) / kMcChunk), row_ints(kCnt + 2 * static_cast<size_t>((S + kMcChunk - 1) / kMcChunk)) {}
+};
+
+__device__ __forceinline__ int mc_row_n(int row, int T_chunk, int S, int m, int row0, const int32_t* q_pos0) {
+  const int bi = row / T_chunk;
+  const int r = row - bi * T_chunk;
+  long long nv = (static_cast<long long>(q_pos0[bi]) + row0 + r + 1) / m;
+  if (nv > S) nv = S;
+  if (nv < 0) nv = 0;
+  return static_cast<int>(nv);
+}
+
+// Descending bin search over a shared histogram of NB bins: returns (bin, count
+// of keys in higher bins) for the bin holding the krem-th largest key.
+template <int NB>
+__device__ __forceinline__ void mc_find_bin(const int* h, int krem, int* wsum, int* out_bin, int* out_above) {
+  constexpr int PER = (NB + kMcThreads - 1) / kMcThreads;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int c[PER], tot = 0;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const int d = NB - 1 - PER * tid - q;
+    c[q] = d >= 0 ? h[d] : 0;
+    tot += c[q];
+  }
+  const int inc = warp_incl_scan(tot);
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  int above = inc - tot;
+#pragma unroll
+  for (int w = 0; w < kMcWarps; ++w) above += (w < warp) ? wsum[w] : 0;
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    if (above < krem && krem <= above + c[q]) {
+      *out_bin = NB - 1 - PER * tid - q;
+      *out_above = above;
+    }
+    above += c[q];
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kMcThreads) topk_mc_hist1(const __nv_bfloat16* __restrict__ score, int T_chunk,
+                                                            int S, int ld, int k, int m, int row0,
+                                                            const int32_t* __restrict__ q_pos0, int* __restrict__ ws) {
+  using KO = KeyOf<__nv_bfloat16>;
+  __shared__ int h[kMcHist1];
+  const McLayout L(S);
+  const int row = blockIdx.x / L.C, c = blockIdx.x % L.C;
+  const int n = mc_row_n(row, T_chunk, S, m, row0, q_pos0);
+  if (n <= k) return;
+  const int i0 = c * kMcChunk, i1 = min(n, i0 + kMcChunk);
+  if (i0 >= i1) return;
+  for (int i = threadIdx.x; i < kMcHist1; i += kMcThreads) h[i] = 0;
+  __syncthreads();
+  const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
+  for (int i = i0 + threadIdx.x; i < i1; i += kMcThreads) atomicAdd(&h[KO::get(srow[i]) >> 5], 1);
+  __syncthreads();
+  int* g = ws + static_cast<size_t>(row) * L.row_ints;
+  for (int i = threadIdx.x; i < kMcHist1; i += kMcThreads)
+    if (h[i]) atomicAdd(&g[i], h[i]);
+}
+
+__global__ void __launch_bounds__(kMcThreads) topk_mc_hist2(const __nv_bfloat16* __restrict__ score, int T_chunk,
+                                                            int S, int ld, int k, int m, int row0,
+                                                            const int32_t* __restrict__ q_pos0, int* __restrict__ ws) {
+  using KO = KeyOf<__nv_bfloat16>;
+  __shared__ int h[kMcHist1];
+  __shared__ int h2[kMcHist2];
+  __shared__ int wsum[kMcWarps];
+  __shared__ int s_bin, s_above;
+  const McLayout L(S);
+  const int row = blockIdx.x / L.C, c = blockIdx.x % L.C;
+  const int n = mc_row_n(row, T_chunk, S, m, row0, q_pos0);
+  if (n <= k) return;
+  int* g = ws + static_cast<size_t>(row) * L.row_ints;
+  for (int i = threadIdx.x; i < kMcHist1; i += kMcThreads) h[i] = g[i];
+  if (threadIdx.x < kMcHist2) h2[threadIdx.x] = 0;
+  __syncthreads();
+  mc_find_bin<kMcHist1>(h, k, wsum, &s_bin, &s_above);
+  const int b1 = s_bin;
+  if (c == 0 && threadIdx.x == 0) {
+    g[McLayout::kState + 0] = b1;
+    g[McLayout::kState + 1] = s_above;
+  }
+  const int i0 = c * kMcChunk, i1 = min(n, i0 + kMcChunk);
+  const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
+  for (int i = i0 + threadIdx.x; i < i1; i += kMcThreads) {
+    const uint32_t key = KO::get(srow[i]);
+    if (static_cast<int>(key >> 5) == b1) atomicAdd(&h2[key & 31], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x < kMcHist2 && h2[threadIdx.x]) atomicAdd(&g[McLayout::kHist2 + threadIdx.x], h2[threadIdx.x]);
+}
+
+__global__ void __launch_bounds__(kMcThreads) topk_mc_count(const __nv_bfloat16* __restrict__ score, int T_chunk,
+                                                            int S, int ld, int k, int m, int row0,
+                                                            const int32_t* __restrict__ q_pos0, int* __restrict__ ws) {
+  using KO = KeyOf<__nv_bfloat16>;
+  __shared__ int h2[kMcHist2];
+  __shared__ int wsum[kMcWarps];
+  __shared__ int s_bin, s_above;
+  __shared__ int wc[kMcWarps][2];
+  const McLayout L(S);
+  const int row = blockIdx.x / L.C, c = blockIdx.x % L.C;
+  const int n = mc_row_n(row, T_chunk, S, m, row0, q_pos0);
+  if (n <= k) return;
+  int* g = ws + static_cast<size_t>(row) * L.row_ints;
+  if (threadIdx.x < kMcHist2) h2[threadIdx.x] = g[McLayout::kHist2 + threadIdx.x];
+  __syncthreads();
+  const int b1 = g[McLayout::kState + 0];
+  const int krem1 = k - g[McLayout::kState + 1];
+  mc_find_bin<kMcHist2>(h2, krem1, wsum, &s_bin, &s_above);
+  const uint32_t K = (static_cast<uint32_t>(b1) << 5) | static_cast<uint32_t>(s_bin);
+  const int krem = krem1 - s_above;
+  if (c == 0 && threadIdx.x == 0) {
+    g[McLayout::kState + 2] = static_cast<int>(K);
+    g[McLayout::kState + 3] = krem;
+  }
+  const int i0 = c * kMcChunk, i1 = min(n, i0 + kMcChunk);
+  const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
+  int n_gt = 0, n_eq = 0;
+  for (int i = i0 + threadIdx.x; i < i1; i += kMcThreads) {
+    const uint32_t key = KO::get(srow[i]);
+    n_gt += key > K;
+    n_eq += key == K;
+  }
+  n_gt = __reduce_add_sync(0xffffffffu, n_gt);
+  n_eq = __reduce_add_sync(0xffffffffu, n_eq);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) { wc[warp][0] = n_gt; wc[warp][1] = n_eq; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int a = 0, b = 0;
+    for (int w = 0; w < kMcWarps; ++w) { a += wc[w][0]; b += wc[w][1]; }
+    g[McLayout::kCnt + 2 * c] = a;
+    g[McLayout::kCnt + 2 * c + 1] = b;
+  }
+}
+
+__global__ void __launch_bounds__(kMcThreads) topk_mc_emit(const __nv_bfloat16* __restrict__ score, int T_chunk,
+                                                           int S, int ld, int k, int m, int row0,
+                                                           const int32_t* __restrict__ q_pos0,
+                                                           const int* __restrict__ ws, int32_t* __restrict__ idx) {
+  using KO = KeyOf<__nv_bfloat16>;
+  __shared__ int wcnt[kMcWarps][2];
+  const McLayout L(S);
+  const int row = blockIdx.x / L.C, c = blockIdx.x % L.C;
+  const int n = mc_row_n(row, T_chunk, S, m, row0, q_pos0);
+  int32_t* out = idx + static_cast<size_t>(row) * k;
+  const int i0 = c * kMcChunk;
+  if (n <= k) {
+    // every visible entry, then -1 pads; chunk c covers output slots [i0, i0 + kMcChunk)
+    const int hi = c == L.C - 1 ? k : min(k, i0 + kMcChunk);   // the last chunk also covers slots >= S
+    for (int i = i0 + threadIdx.x; i < hi; i += kMcThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  const int i1 = min(n, i0 + kMcChunk);
+  if (i0 >= i1) return;
+  const int* g = ws + static_cast<size_t>(row) * L.row_ints;
+  const uint32_t K = static_cast<uint32_t>(g[McLayout::kState + 2]);
+  const int krem = g[McLayout::kState + 3];
+  int out_pos = 0, eq_before = 0;
+  for (int cc = 0; cc < c; ++cc) {
+    const int gt = g[McLayout::kCnt + 2 * cc], eq = g[McLayout::kCnt + 2 * cc + 1];
+    out_pos += gt + max(0, min(eq, krem - eq_before));
+    eq_before += eq;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
+  const int seg = kMcChunk / kMcWarps;
+  const int s0 = i0 + warp * seg, s1 = min(i1, s0 + seg);
+  int n_gt = 0, n_eq = 0;
+  for (int b0 = s0; b0 < s1; b0 += 32) {
+    const int i = b0 + lane;
+    const uint32_t key = i < s1 ? static_cast<uint32_t>(KO::get(srow[i])) : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, i < s1 && key > K));
+    n_eq += __popc(__ballot_sync(0xffffffffu, i < s1 && key == K));
+  }
+  if (lane == 0) { wcnt[warp][0] = n_gt; wcnt[warp][1] = n_eq; }
+  __syncthreads();
+  for (int w = 0; w < warp; ++w) {
+    out_pos += wcnt[w][0] + max(0, min(wcnt[w][1], krem - eq_before));
+    eq_before += wcnt[w][1];
+  }
+  const unsigned below = (1u << lane) - 1u;
+  for (int b0 = s0; b0 < s1; b0 += 32) {
+    const int i = b0 + lane;
+    const uint32_t key = i < s1 ? static_cast<uint32_t>(KO::get(srow[i])) : 0u;
+    const bool gt = i < s1 && key > K;
+    const bool eq = i < s1 && key == K;
+    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_before + __popc(eqm & below) < krem);
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[out_pos + __popc(tm & below)] = i;
+    out_pos += __popc(tm);
+    eq_before += __popc(eqm);
+  }
+}
+
+inline bool topk_use_multi(int score_dtype, long long rows, int S) {
+  return score_dtype == CSA_BF16 && rows <= kMcRowsMax && S >= kMcMinS;
+}
+
+inline size_t topk_multi_bytes(long long rows, int S) {
+  return static_cast<size_t>(rows) * McLayout(S).row_ints * sizeof(int);
+}
+
+int launch_topk_multi(const __nv_bfloat16* score, long long rows, int T_chunk, int S, int ld, int k, int m, int row0,
+                      const int32_t* q_pos0, int32_t* idx, int* ws, cudaStream_t st) {
+  const McLayout L(S);
+  cudaError_t e = cudaMemsetAsync(ws, 0, topk_multi_bytes(rows, S), st);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  const unsigned grid = static_cast<unsigned>(rows * L.C);
+  topk_mc_hist1<<<grid, kMcThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, ws);
+  topk_mc_hist2<<<grid, kMcThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, ws);
+  topk_mc_count<<<grid, kMcThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, ws);
+  topk_mc_emit<<<grid, kMcThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, ws, idx);
+  return check_launch();
+}
+
 template <typename T>
 int launch_topk(const T* score, int B, int T_chunk, int S, int ld, int k, int m, int row0, const int32_t* q_pos0,
                 int32_t* idx, cudaStream_t st) {
@@ -224,15 +472,17 @@ using namespace csa;
 extern "C" {
 
 size_t topk_workspace_size(int B, int T_chunk, int S, int k) {
-  (void)B; (void)T_chunk; (void)S; (void)k;
-  return 0;
+  (void)k;
+  if (B <= 0 || T_chunk <= 0 || S <= 0) return 0;
+  const long long rows = static_cast<long long>(B) * T_chunk;
+  return topk_use_multi(CSA_BF16, rows, S) ? topk_multi_bytes(rows, S) : 0;
 }
 
 int topk_select(const void* score, int score_dtype, int B, int T_chunk, int S, int score_ld, int k, int m,
                 int row0, const int32_t* q_pos0, int32_t* idx, void* workspace, size_t ws_bytes,
                 csa_stream_t stream) {
-  (void)workspace; (void)ws_bytes;
   CSA_REQUIRE(score && idx && q_pos0, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 3) == 0, CSA_ERR_ALIGNMENT);
   CSA_REQUIRE(B >= 0 && T_chunk >= 0 && S >= 0 && score_ld >= S && k >= 1 && m >= 1 && row0 >= 0,
               CSA_ERR_INVALID_ARG);
   CSA_REQUIRE(score_dtype == CSA_F32 || score_dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
@@ -240,6 +490,9 @@ int topk_select(const void* score, int score_dtype, int B, int T_chunk, int S, i
   if (rows == 0) return CSA_OK;
   CSA_REQUIRE(rows < (1ll << 31), CSA_ERR_UNSUPPORTED);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (topk_use_multi(score_dtype, rows, S) && workspace != nullptr && ws_bytes >= topk_multi_bytes(rows, S))
+    return launch_topk_multi(static_cast<const __nv_bfloat16*>(score), rows, T_chunk, S, score_ld, k, m, row0,
+                             q_pos0, idx, static_cast<int*>(workspace), st);
   if (score_dtype == CSA_F32)
     return launch_topk(static_cast<const float*>(score), B, T_chunk, S, score_ld, k, m, row0, q_pos0, idx, st);
   return launch_topk(static_cast<const __nv_bfloat16*>(score), B, T_chunk, S, score_ld, k, m, row0, q_pos0, idx,

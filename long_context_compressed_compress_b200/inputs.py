@@ -79,7 +79,7 @@ def decode_state(cfg, device="cpu", extra_entries=None):
     block (the compressor carry).  Capacity leaves room for ``extra_entries``
     entries emitted during decoding.
 
-    Order: kv_c, k_I_src, ring, carry a, b, z, a_I, b_I, z_I.
+    Order: kv_c, k_I_src, ring, carry a, b, z, a_I, b_I, z_I, sink [H].
     """
     gen = torch.Generator(device=device)
     gen.manual_seed(cfg.seed)
@@ -95,6 +95,7 @@ def decode_state(cfg, device="cpu", extra_entries=None):
     st["ring"] = _draw(gen, (B, cfg.W, D), device, dt)
     for name, dim in (("a", D), ("b", D), ("z", D), ("a_I", DI), ("b_I", DI), ("z_I", DI)):
         st["carry_" + name] = _draw(gen, (B, m, dim), device, dt)
+    st["sink"] = _draw(gen, (cfg.H,), device, torch.float32)
     return st
 
 

@@ -111,3 +111,121 @@ class HcaPrefill:
             ops.hca_dense_attn_fwd(x["q"], self.kv_c, x["kv_raw"], x["sink"], c.tau, c.W, self.q_pos0, self.out,
                                    c.m, lse=self.lse)
         return self.out
+
+
+_CARRY = ("a", "b", "z", "a_I", "b_I", "z_I")
+
+
+class CsaDecode:
+    """Buffers + call sequence of one CSA decode step: one new token for each of
+    B sequences (cf-1.com/news/5231315 §3.1, §3.3; the cached state grows by one
+    compressed entry every m tokens and the raw window is a W-slot ring).
+
+    ``state`` is the synthetic cache at position T0 (``inputs.decode_state`` on
+    the device): kv_c [B, cap, D], k_I_src [B, cap, D_I], ring [B, W, D] and the
+    raw rows of the last complete block ``carry_*`` [B, m, dim].  The indexer keys
+    of the cache are quantised to NVFP4 once here; per step:
+
+        csa_ring_append x6            token p -> compressor carry slot p % 2m
+        csa_compress (decode mode)    entry (p+1)/m - 1 when block completes -> kv_c
+        csa_compress (decode, NVFP4)  the same entry's indexer key        -> k_I
+        csa_ring_append               token p's raw KV -> ring slot p % W
+        nvfp4_quantize                q_I
+        indexer_score                 score [B, 1, cap] (visible prefix only)
+        topk_select                   idx [B, 1, k] (multi-CTA rows, workspace)
+        sparse_attn_fwd               out [B, 1, H, D] (window + sink fused)
+        csa_pos_advance               p += 1 on the device
+
+    Every launch reads the position from device memory, so the step can be
+    captured once in a CUDA graph (``capture``) and replayed.
+    """
+
+    def __init__(self, cfg, state, T0, device="cuda", gscale=1.0, with_lse=False):
+        self.cfg = c = cfg
+        dt = _DT[c.dtype]
+        self.dt = dt
+        self.g = gscale
+        self.T0 = T0
+        self.kv_c = state["kv_c"]
+        B, cap, D = self.kv_c.shape
+        self.cap = cap
+        self.k_fp4 = torch.empty((B, cap, c.DI // 2), dtype=torch.uint8, device=device)
+        self.k_sf = torch.empty((B, cap, c.DI // 16), dtype=torch.uint8, device=device)
+        ops.nvfp4_quantize(state["k_I_src"], self.k_fp4, self.k_sf, gscale)
+        self.ring = state["ring"]
+        self.carry = {}
+        slot0 = ((T0 // c.m - 1) % 2) * c.m      # the last complete block's slots
+        for n in _CARRY:
+            src = state["carry_" + n]
+            buf = torch.zeros((B, 2 * c.m, src.shape[-1]), dtype=dt, device=device)
+            buf[:, slot0:slot0 + c.m] = src
+            self.carry[n] = buf
+        self.pos = torch.full((B,), T0, dtype=torch.int32, device=device)
+        self.q_fp4 = torch.empty((B, 1, c.HI, c.DI // 2), dtype=torch.uint8, device=device)
+        self.q_sf = torch.empty((B, 1, c.HI, c.DI // 16), dtype=torch.uint8, device=device)
+        sdt = torch.float32 if c.dtype == "f32" else torch.bfloat16
+        self.score = torch.empty((B, 1, cap), dtype=sdt, device=device)
+        self.idx = torch.empty((B, 1, c.k), dtype=torch.int32, device=device)
+        self.out = torch.empty((B, 1, c.H, D), dtype=dt, device=device)
+        self.lse = torch.empty((B, 1, c.H), dtype=torch.float32, device=device) if with_lse else None
+        nws = ops.topk_workspace_size(B, 1, cap, c.k)
+        self.ws = torch.empty((max(1, nws // 4),), dtype=torch.int32, device=device) if nws else None
+        self.sink = state.get("sink")
+        self.launches = 6 + 2 + 1 + 1 + 1 + (5 if nws else 1) + 1 + 1
+        self.graph = None
+        self.x = None
+
+    def step(self, x, timer=None):
+        """x: per-step device inputs (``inputs.decode_step_inputs`` layout, plus
+        ``sink`` [H] if the state has none).  Returns out [B, 1, H, D]."""
+        c = self.cfg
+        t = timer or _no_timer
+        for n in _CARRY:
+            with t("csa_ring_append"):
+                ops.csa_ring_append(x[n], self.carry[n], self.pos)
+        with t("csa_compress"):
+            ops.csa_compress(self.carry["a"], self.carry["b"], self.carry["z"], c.m, out=self.kv_c,
+                             ring_pos=self.pos, out_bstride=self.cap)
+        with t("csa_compress_indexer_keys"):
+            ops.csa_compress(self.carry["a_I"], self.carry["b_I"], self.carry["z_I"], c.m, out_fp4=self.k_fp4,
+                             out_sf=self.k_sf, gscale=self.g, ring_pos=self.pos, out_bstride=self.cap,
+                             out_dtype=self.dt)
+        with t("csa_ring_append"):
+            ops.csa_ring_append(x["kv_raw"], self.ring, self.pos)
+        with t("nvfp4_quantize"):
+            ops.nvfp4_quantize(x["q_I"], self.q_fp4, self.q_sf, self.g)
+        with t("indexer_score"):
+            ops.indexer_score(self.q_fp4, self.q_sf, self.k_fp4, self.k_sf, x["w"].view(-1, 1, c.HI), self.pos,
+                              self.score, self.cap, c.m, q_gscale=self.g, k_gscale=self.g)
+        with t("topk_select"):
+            ops.topk_select(self.score, self.idx, self.cap, c.m, self.pos, workspace=self.ws)
+        sink = x["sink"] if "sink" in x else self.sink
+        with t("sparse_attn_fwd"):
+            ops.sparse_attn_fwd(x["q"].view(-1, 1, c.H, x["q"].shape[-1]), self.kv_c, self.idx, self.ring, sink,
+                                c.tau, c.W, self.pos, self.out, self.lse, raw_cap=c.W)
+        with t("csa_pos_advance"):
+            ops.csa_pos_advance(self.pos, 1)
+        return self.out
+
+    def capture(self, x):
+        """Record one step on static input buffers ``x`` into a CUDA graph; the
+        caller refills ``x`` in place and calls ``replay``.  Run ``step`` once
+        before capturing (first-call set-up such as kernel attributes must not
+        happen inside the capture), and note that capture itself does not
+        advance the position."""
+        self.x = x
+        p0 = self.pos.clone()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                self.step(x)
+        torch.cuda.current_stream().wait_stream(s)
+        self.pos.copy_(p0)
+        self.graph = g
+        return g
+
+    def replay(self):
+        self.graph.replay()
+        return self.out

@@ -37,7 +37,7 @@ Where those pages leave a formula open, the oracle takes these readings
   * Attention: MQA, one shared KV head, key = value = the entry (or raw token)
     vector; the sliding window holds raw tokens j with p-W < j <= p, j >= 0
     ([cf-1] §3.3, W = 128); the sink logit sigma_h adds exp(sigma_h) to the
-    softmax denominator only ([cf-1] §3.3 "可学习的分母加项").
+    softmax denominator only ([cf-1] §3.3: a learnable term added to the denominator).
     lse is the log-sum-exp of the logits without the sink.
 """
 from __future__ import annotations
@@ -50,7 +50,7 @@ __all__ = [
     "csa_compress", "hca_compress", "nvfp4_quantize", "visible_entries",
     "indexer_score", "round_scores", "topk_select", "attend_rows",
     "sparse_attn", "dense_attn", "swa_sink_merge", "round_out",
-    "csa_layer", "hca_layer",
+    "csa_layer", "hca_layer", "csa_decode_step",
 ]
 
 
@@ -70,8 +70,8 @@ def _f64(x):
 # ---------------------------------------------------------------------------
 
 def csa_compress(a, b, z, m: int = 4, first_has_pred: bool = False):
-    """Overlapping gated m:1 compression ([cf-1] §3.1; [yfxerp] §1, "每 4 个相邻 Token
-    的 KV 压缩成 1 个条目"; kv_compress_ratio 4 in the [attention.csa] block).
+    """Overlapping gated m:1 compression ([cf-1] §3.1; [yfxerp] §1: the KV of every
+    4 adjacent tokens becomes one entry; kv_compress_ratio 4 in the [attention.csa] block).
 
     a, b, z: [..., T, D].  Returns e: [..., S, D] float64 (unrounded), where
     S = T // m, or T // m - 1 when ``first_has_pred`` (then rows [0, m) are only
@@ -109,8 +109,8 @@ def csa_compress(a, b, z, m: int = 4, first_has_pred: bool = False):
 
 
 def hca_compress(a, z, m: int = 128):
-    """Non-overlapping gated m:1 pooling ([cf-1] §3.2, "每 128 个 token 压缩成 1 个
-    entry"; compress_ratio 128 in the [attention.hca] block of [yfxerp] §3).
+    """Non-overlapping gated m:1 pooling ([cf-1] §3.2: one entry per 128 tokens;
+    compress_ratio 128 in the [attention.hca] block of [yfxerp] §3).
 
     e[i,c] = sum_{t in block i} softmax_{t in block i}(z[t,c]) * a[t,c]
     """
@@ -131,8 +131,8 @@ def hca_compress(a, z, m: int = 128):
 # ---------------------------------------------------------------------------
 
 def nvfp4_quantize(x, g: float = 1.0):
-    """NVFP4 block quantisation along the last dim, blocks of 16 ([cf-1] §3.4 "QK 计算
-    直接用 FP4 精度", §4.4 FP4 QK path; 16-element blocks with E4M3 scales).
+    """NVFP4 block quantisation along the last dim, blocks of 16 ([cf-1] §3.4: the
+    indexer's QK runs in FP4; §4.4 FP4 QK path; 16-element blocks with E4M3 scales).
 
     For block j with amax_j = max |x| (x taken as fp32):
         s_j  = E4M3_rne_sat( fp32( amax_j / fp32(6*g) ) )
@@ -196,15 +196,15 @@ def indexer_score(qhat, khat, w, positions, m: int):
 
 def round_scores(score, dtype: str):
     """Round exact scores once to the stored type: 'f32' or 'bf16' (RNE); the
-    index scores are stored in BF16 ([cf-1] §4.4 "index score 从 FP32 量化到 BF16")."""
+    index scores are stored in BF16 ([cf-1] §4.4: the score is narrowed from FP32 to BF16)."""
     return formats.bf16(score) if dtype == "bf16" else formats.f32(score)
 
 
 def topk_select(score, positions, m: int, k: int):
     """Per row, the k largest visible scores; ties go to the smaller entry index;
     indices are emitted ascending and padded with -1.  If fewer than k entries are
-    visible, all of them are returned ([cf-1] §3.1 "每个 query ... 选 top-k 个压缩
-    entry"; top_k_blocks in the [attention.csa] block of [yfxerp] §3).
+    visible, all of them are returned ([cf-1] §3.1: each query picks its top-k
+    compressed entries; top_k_blocks in the [attention.csa] block of [yfxerp] §3).
 
     score [B,T,S] (values as stored, compared exactly; +0 and -0 are equal).
     Returns int32 [B,T,k].
@@ -291,7 +291,7 @@ def sparse_attn(q, kv_c, idx, kv_raw, raw_cap, sink, tau, W, positions, rows=Non
 
 def dense_attn(q, kv_c, kv_raw, raw_cap, sink, tau, W, positions, m, rows=None):
     """HCA attention: each query attends to every visible compressed entry
-    ("不做稀疏选择，直接 dense attention", [cf-1] §3.2) plus the raw window and sink."""
+    ([cf-1] §3.2: no sparse selection, dense attention) plus the raw window and sink."""
     q, kv_c, kv_raw = _f64(q), _f64(kv_c), _f64(kv_raw)
     H = q.shape[2]
     snk = np.full(H, -np.inf) if sink is None else _f64(sink)
@@ -401,3 +401,49 @@ def hca_layer(x, m, W, tau, dtype, rows=None, return_all=False):
     if return_all:
         res["kv_c"] = kv_c
     return res
+
+
+# ---------------------------------------------------------------------------
+# Decode (one new token per sequence).  cf-1.com/news/5231315 §3.1/§3.3: the
+# compressed cache grows by one entry per m tokens, the raw window keeps the
+# last W tokens.  Order of a step at position p: append token p's raw rows to
+# the compressor carry (slot p mod 2m); if block (p+1)/m - 1 just completed,
+# emit its entry (current block = a rows, predecessor = b rows) into the cache
+# before scoring; write token p's raw KV into ring slot p mod W; then score,
+# select and attend for the single query, exactly as in prefill.
+# ---------------------------------------------------------------------------
+def csa_decode_step(st, x, p, m, k, W, tau, dtype, gscale=1.0):
+    """One decode step for every sequence at common position ``p``.
+
+    ``st`` (updated in place) holds float64 arrays: ``kv_c`` [B,S,D] and ``khat``
+    [B,S,DI] (the cache, S = entries emitted so far), ``ring`` [B,W,D], and the
+    carry rings ``carry_<a|b|z|a_I|b_I|z_I>`` [B,2m,dim].  ``x`` holds the step's
+    inputs q [B,H,D], q_I [B,HI,DI], w [B,HI], and the new token's a, b, z, a_I,
+    b_I, z_I, kv_raw rows.  Returns out [B,H,D] (rounded to ``dtype``), lse
+    [B,H], idx [B,k] and the bf16/f32-rounded score [B,S]."""
+    for name in ("a", "b", "z", "a_I", "b_I", "z_I"):
+        st["carry_" + name][:, p % (2 * m)] = _f64(x[name])
+    if (p + 1) % m == 0:
+        i = (p + 1) // m - 1
+        assert st["kv_c"].shape[1] == i, "cache length must equal the entry being emitted"
+        cur = slice((i % 2) * m, (i % 2) * m + m)
+        prev = slice(((i + 1) % 2) * m, ((i + 1) % 2) * m + m)
+
+        def entry(a, b, z):
+            slab = [np.concatenate([st["carry_" + n][:, prev], st["carry_" + n][:, cur]], axis=1) for n in (a, b, z)]
+            return round_out(csa_compress(slab[0], slab[1], slab[2], m, first_has_pred=True), dtype)
+
+        st["kv_c"] = np.concatenate([st["kv_c"], entry("a", "b", "z")], axis=1)
+        e_I = entry("a_I", "b_I", "z_I")
+        st["khat"] = np.concatenate([st["khat"], nvfp4_quantize(e_I, gscale)["xhat"]], axis=1)
+    st["ring"][:, p % W] = _f64(x["kv_raw"])
+    q = _f64(x["q"])[:, None]                      # [B,1,H,D]
+    B = q.shape[0]
+    pos = np.full((B, 1), p, dtype=np.int64)
+    qhat = nvfp4_quantize(_f64(x["q_I"])[:, None], gscale)["xhat"]
+    sc = indexer_score(qhat, st["khat"], _f64(x["w"])[:, None], pos, m)
+    sc = round_scores(sc, "f32" if dtype == "f32" else "bf16")
+    idx = topk_select(sc, pos, m, k)
+    out, lse = sparse_attn(q, st["kv_c"], idx, st["ring"], W, x["sink"], tau, W, pos)
+    return {"out": round_out(out, dtype)[:, 0], "lse": formats.f32(lse)[:, 0], "idx": idx[:, 0],
+            "score": sc[:, 0]}

@@ -240,6 +240,35 @@ def test_topk_long_rows_all_equal(ops):
     np.testing.assert_array_equal(idx.cpu().numpy()[0, 0], np.arange(k))
 
 
+@pytest.mark.parametrize("k", [64, 1024, 9000])
+def test_topk_multi_cta_rows(ops, k):
+    """Few long BF16 rows run split across CTAs through the workspace; the
+    result equals the oracle and the one-CTA-per-row path, on repeated calls
+    with a workspace that starts out holding garbage."""
+    B, T, m, S = 3, 4, 4, 40000
+    g = torch.Generator().manual_seed(k + 7)
+    sc = torch.randn((B, T, S), generator=g)
+    sc[0, 1] = torch.relu(sc[0, 1])                      # many zeros
+    sc[1, 0] = torch.round(sc[1, 0] * 4) / 4             # many ties
+    sc[1, 2] = 1.5                                       # all equal
+    sc[2, 3, ::7] = -0.0
+    sc = sc.to(torch.bfloat16)
+    pos0 = torch.tensor([4 * S, 4 * 20000 + 1, 4 * 1000], dtype=torch.int32)
+    nbytes = ops.topk_workspace_size(B, T, S, k)
+    assert nbytes > 0
+    ws = torch.full((nbytes // 4,), 12345, dtype=torch.int32, device="cuda")
+    pos = np.arange(T)[None] + pos0.numpy()[:, None]
+    ref = oracle.topk_select(_np(sc), pos, m, k)
+    scd, posd = sc.cuda(), pos0.cuda()
+    for _ in range(2):
+        idx = torch.full((B, T, k), -7, dtype=torch.int32, device="cuda")
+        ops.topk_select(scd, idx, S, m, posd, workspace=ws)
+        np.testing.assert_array_equal(idx.cpu().numpy(), ref)
+    idx1 = torch.full((B, T, k), -7, dtype=torch.int32, device="cuda")
+    ops.topk_select(scd, idx1, S, m, posd)
+    np.testing.assert_array_equal(idx1.cpu().numpy(), ref)
+
+
 # -------------------------------------------------------------- attention
 
 def _attn_inputs(B, T, H, D, S, dtype, seed, q_scale=1.0):

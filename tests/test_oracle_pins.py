@@ -160,7 +160,7 @@ def test_e2m1_against_brute_force_including_every_midpoint():
 
 def test_fp4_values_are_exact_in_fp8_lossless_dequant():
     """Every E2M1 value is an E4M3 value, so FP4 -> FP8 dequantisation is exact,
-    as cf-1.com/news/5231315 §4.4 states ("FP4 到 FP8 的反量化是无损的")."""
+    as cf-1.com/news/5231315 §4.4 says (dequantising FP4 to FP8 loses nothing)."""
     g = formats.E2M1_VALUES
     np.testing.assert_array_equal(formats.e4m3(np.concatenate([g, -g])), np.concatenate([g, -g]))
 
@@ -395,3 +395,33 @@ def test_bf16_rounding_matches_torch_on_fp32_inputs():
     x = (RNG.standard_normal(100000) * np.exp(RNG.uniform(-20, 20, 100000))).astype(np.float32)
     ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(formats.bf16(x.astype(np.float64)), ref)
+
+
+def test_decode_steps_equal_prefill_rows():
+    """Decoding token p from a cache built from tokens [0, T0) gives row p of a
+    prefill over the same tokens: pins the decode step's carry slots, emission
+    timing (entry (p+1)/m - 1 visible at step p), NVFP4 keys and ring window."""
+    from long_context_compressed_compress_b200 import configs, inputs
+    cfg = configs.scaled(configs.PR1, T=96, k=8)
+    m, W, T0 = cfg.m, 16, 64
+    x = inputs.layer_inputs(cfg, device="cpu")
+    full = oracle.csa_layer(x, m, cfg.k, W, cfg.tau, cfg.dtype)
+    f = {k: v.to(torch.float64).numpy() for k, v in x.items()}
+    st = {"kv_c": oracle.round_out(oracle.csa_compress(f["a"][:, :T0], f["b"][:, :T0], f["z"][:, :T0], m), "f32"),
+          "ring": np.zeros((cfg.B, W, cfg.D))}
+    k_src = oracle.round_out(oracle.csa_compress(f["a_I"][:, :T0], f["b_I"][:, :T0], f["z_I"][:, :T0], m), "f32")
+    st["khat"] = oracle.nvfp4_quantize(k_src)["xhat"]
+    for j in range(T0 - W, T0):
+        st["ring"][:, j % W] = f["kv_raw"][:, j]
+    for n in ("a", "b", "z", "a_I", "b_I", "z_I"):
+        c = np.zeros((cfg.B, 2 * m, f[n].shape[-1]))
+        for j in range(T0 - m, T0):
+            c[:, j % (2 * m)] = f[n][:, j]
+        st["carry_" + n] = c
+    for p in range(T0, cfg.T):
+        xs = {n: f[n][:, p] for n in ("q", "q_I", "w", "a", "b", "z", "a_I", "b_I", "z_I", "kv_raw")}
+        xs["sink"] = f["sink"]
+        r = oracle.csa_decode_step(st, xs, p, m, cfg.k, W, cfg.tau, cfg.dtype)
+        np.testing.assert_array_equal(r["idx"][0], full["idx"][p])     # rows are (b, t), B = 1
+        np.testing.assert_allclose(r["out"][0], full["out"][p], rtol=1e-12, atol=1e-12)
+    assert st["kv_c"].shape[1] == cfg.T // m
