@@ -172,6 +172,26 @@ int topk_select(const void* score, int score_dtype, int B, int T_chunk, int S,
 size_t topk_workspace_size(int B, int T_chunk, int S, int k);
 
 /*
+ * topk_select_noalloc -- topk_select for callers that cannot allocate device
+ * memory (no workspace argument).  The pages have no counterpart to this call;
+ * it exists only for allocator-free callers.  Same arguments, layouts, result
+ * and statuses as topk_select with a workspace, except:
+ *   - scratch: the multi-CTA path uses a fixed 1 MiB array inside the library
+ *     (one per device per process) instead of caller memory; the call itself
+ *     allocates nothing.  A shape whose multi-CTA histograms need more than
+ *     1 MiB (topk_workspace_size() > 1048576) returns CSA_ERR_UNSUPPORTED and
+ *     queues no work.  Shapes needing no scratch run the one-CTA-per-row path.
+ *   - concurrency: calls that overlap in time on the same device (other
+ *     streams, other host threads) share that scratch and race; order them.
+ *   - set-up: the first call on a device (with that device current) looks up
+ *     the scratch address; make it before any stream capture begins.
+ */
+int topk_select_noalloc(const void* score, int score_dtype, int B, int T_chunk,
+                        int S, int score_ld, int k, int m, int row0,
+                        const int32_t* q_pos0, int32_t* idx,
+                        csa_stream_t stream);
+
+/*
  * sparse_attn_fwd -- CSA attention ([cf-1] §3.1 sparse attention over the
  * selected compressed entries, §3.3 128-token raw window and attention sink).
  * For query row r (position p) and head h, over the key set

@@ -18,6 +18,8 @@
 //
 // One CTA (128 threads) per query row; the visible prefix of the row is staged
 // in shared memory when it fits, otherwise every pass re-reads it from L2.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace csa {
@@ -500,3 +502,83 @@ int topk_select(const void* score, int score_dtype, int B, int T_chunk, int S, i
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// topk_select_noalloc: the same selection for callers that may not allocate
+// device memory.  An allocator-free caller (a real-time serving loop that
+// must not block on the CUDA allocator, a host runtime that hands the library
+// no memory of its own, code running where a cudaMalloc could implicitly
+// synchronise the device) cannot provide the multi-CTA workspace.  This entry
+// uses a fixed scratch array that lives in the library's own device image
+// instead, so it allocates nothing, ever: no cudaMalloc, no cudaFree, no
+// library routine that allocates.
+//
+// Limits and rules, in plain words:
+//   * the scratch holds kNoAllocScratchBytes (1 MiB); a shape whose multi-CTA
+//     histograms need more is rejected with CSA_ERR_UNSUPPORTED before any
+//     work is queued (32 rows of 262,144 entries need about 275 KB);
+//   * the scratch is one per device and per process: two calls that overlap
+//     in time on the same device (different streams, or different host
+//     threads) race on it and give wrong results;
+//   * the first call on each device looks up the scratch's device address
+//     (cudaGetSymbolAddress with that device current); make that first call
+//     before any stream capture begins;
+//   * shapes that need no scratch run the one-CTA-per-row kernel, as
+//     topk_select does without a workspace.
+// ---------------------------------------------------------------------------
+namespace csa {
+
+constexpr size_t kNoAllocScratchBytes = 1u << 20;
+static __device__ __align__(256) uint8_t g_topk_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
+
+// Device address of this device's scratch (set-up on first use per device).
+static int noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_cuda_error(e);
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return CSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_topk_scratch);
+    if (e != cudaSuccess) return set_cuda_error(e);
+    if (p == nullptr) return CSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return CSA_OK;
+}
+
+}  // namespace csa
+
+extern "C" int topk_select_noalloc(const void* score, int score_dtype, int B, int T_chunk, int S, int score_ld,
+                                   int k, int m, int row0, const int32_t* q_pos0, int32_t* idx,
+                                   csa_stream_t stream) {
+  CSA_REQUIRE(score && idx && q_pos0, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(B >= 0 && T_chunk >= 0 && S >= 0 && score_ld >= S && k >= 1 && m >= 1 && row0 >= 0,
+              CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(score_dtype == CSA_F32 || score_dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
+  const long long rows = static_cast<long long>(B) * T_chunk;
+  if (rows == 0) return CSA_OK;
+  CSA_REQUIRE(rows < (1ll << 31), CSA_ERR_UNSUPPORTED);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!topk_use_multi(score_dtype, rows, S)) {
+    if (score_dtype == CSA_F32)
+      return launch_topk(static_cast<const float*>(score), B, T_chunk, S, score_ld, k, m, row0, q_pos0, idx, st);
+    return launch_topk(static_cast<const __nv_bfloat16*>(score), B, T_chunk, S, score_ld, k, m, row0, q_pos0,
+                       idx, st);
+  }
+  // the multi-CTA histograms must fit the fixed scratch; larger shapes are refused
+  CSA_REQUIRE(topk_multi_bytes(rows, S) <= kNoAllocScratchBytes, CSA_ERR_UNSUPPORTED);
+  void* scratch = nullptr;
+  const int r = noalloc_scratch(&scratch);
+  if (r != CSA_OK) return r;
+  // launch_topk_multi clears the histogram region it uses (cudaMemsetAsync,
+  // which allocates nothing) before its first kernel
+  return launch_topk_multi(static_cast<const __nv_bfloat16*>(score), rows, T_chunk, S, score_ld, k, m, row0, q_pos0,
+                           idx, static_cast<int*>(scratch), st);
+}

@@ -48,6 +48,7 @@ _SIGS = {
     "indexer_score": ([P, P, F, P, P, F, P, I, I, I, I, I, I, I, I, I, P, P, I, I, P], I),
     "topk_select": ([P, I, I, I, I, I, I, I, I, P, P, P, SZ, P], I),
     "topk_workspace_size": ([I, I, I, I], SZ),
+    "topk_select_noalloc": ([P, I, I, I, I, I, I, I, I, P, P, P], I),
     "sparse_attn_fwd": ([P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, P, P, P, I, P], I),
     "hca_dense_attn_fwd": ([P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, I, P, P, P, I, P], I),
     "swa_sink_merge": ([P, P, P, P, P, F, I, I, I, I, I, I, I, I, P, P, I, P], I),
@@ -137,6 +138,15 @@ def topk_select(score, idx, S, m, q_pos0, row0=0, workspace=None, stream=None):
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("topk_select", lib.topk_select(_ptr(score), _dt(score), B, T_chunk, S, ld, k, m, row0,
                                           _ptr(q_pos0), _ptr(idx), _ptr(workspace), ws, _stream(stream)))
+
+
+def topk_select_noalloc(score, idx, S, m, q_pos0, row0=0, stream=None):
+    """topk_select without a workspace: the library's fixed scratch serves the
+    multi-CTA path (see the C header for its size limit and concurrency rule)."""
+    B, T_chunk, ld = score.shape
+    k = idx.shape[-1]
+    _check("topk_select_noalloc", lib.topk_select_noalloc(_ptr(score), _dt(score), B, T_chunk, S, ld, k, m, row0,
+                                                          _ptr(q_pos0), _ptr(idx), _stream(stream)))
 
 
 def topk_workspace_size(B, T_chunk, S, k):
