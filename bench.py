@@ -48,8 +48,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=0,
                     help="profiling case: override the layer's token count (not a bench line)")
-    ap.add_argument("--workload", default="csa_prefill_32k", choices=["csa_prefill_32k", "csa_decode_32x1m"],
-                    help="csa_prefill_32k (the default line) or csa_decode_32x1m (decode steps/s)")
+    ap.add_argument("--workload", default="csa_prefill_32k", choices=["csa_prefill_32k", "csa_decode_32x1m", "stack_hhcc_256k"],
+                    help="csa_prefill_32k (the default line), csa_decode_32x1m (decode steps/s) or "
+                         "stack_hhcc_256k (4-layer prefill stack tokens/s)")
     return ap.parse_args()
 
 
@@ -152,9 +153,10 @@ class OracleSample:
         import oracle
         from long_context_compressed_compress_b200 import inputs
         self.np, self.oracle, self.cfg = np, oracle, cfg
-        # host inputs converted to float64 once (the oracle's working precision)
-        self.x = {k: v.to(torch_f64()).numpy() for k, v in inputs.layer_inputs(cfg, device="cpu").items()}
-        self.idx = np.full((cfg.B, cfg.T, cfg.k), -1, dtype=np.int32)
+        # host inputs converted to float64 once (the oracle's working precision);
+        # q stays in its storage dtype and the oracle converts the rows it reads
+        self.x = {k: (v if k == "q" else v.to(torch_f64()).numpy())
+                  for k, v in inputs.layer_inputs(cfg, device="cpu").items()}
         self.pos = np.arange(cfg.T)[None]
         self.rng = np.random.default_rng(1234)
         try:
@@ -167,7 +169,6 @@ class OracleSample:
         self.kv = oracle.round_out(oracle.csa_compress(x["a"], x["b"], x["z"], c.m), c.dtype)
         ks = oracle.round_out(oracle.csa_compress(x["a_I"], x["b_I"], x["z_I"], c.m), c.dtype)
         self.khat = oracle.nvfp4_quantize(ks)["xhat"]
-        self.qhat = oracle.nvfp4_quantize(x["q_I"])["xhat"]
         self.t_comp = time.perf_counter() - t0
         self.t_rows = 0.0
         self.n_rows = 0
@@ -179,11 +180,11 @@ class OracleSample:
         for t in ts:
             t = int(t)
             pos = np.array([[t]])
-            sc = o.round_scores(o.indexer_score(self.qhat[:, t:t + 1], self.khat, x["w"][:, t:t + 1], pos, c.m),
+            qhat = o.nvfp4_quantize(x["q_I"][:, t:t + 1])["xhat"]
+            sc = o.round_scores(o.indexer_score(qhat, self.khat, x["w"][:, t:t + 1], pos, c.m),
                                 "bf16" if c.dtype != "f32" else "f32")
             idx = o.topk_select(sc, pos, c.m, c.k)
-            self.idx[0, t] = idx[0, 0]
-            o.sparse_attn(x["q"], self.kv, self.idx, x["kv_raw"], c.T, x["sink"], c.tau, c.W, self.pos,
+            o.sparse_attn(x["q"], self.kv, {(0, t): idx[0, 0]}, x["kv_raw"], c.T, x["sink"], c.tau, c.W, self.pos,
                           rows=[(0, t)])
         dt = time.perf_counter() - t0
         self.t_rows += dt
@@ -262,6 +263,9 @@ def main():
         cfg = configs.scaled(cfg, T=args.T)
     if args.workload == "csa_decode_32x1m":
         main_decode(args, rank, world, local)
+        return
+    if args.workload == "stack_hhcc_256k":
+        main_stack(args, rank, world, local)
         return
     if args.impl == "reference":
         run_reference(args, cfg, rank)
@@ -599,6 +603,167 @@ def main_decode(args, rank, world, local):
     if rank == 0:
         print(json.dumps(line), flush=True)
     lay.graph = None
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def attn_flops(cfg):
+    """4·H·D flops per (query, head, attended row); rows = the selected (CSA) or
+    all visible (HCA) entries plus the raw window, summed over queries."""
+    import numpy as np
+    t = np.arange(cfg.T, dtype=np.int64)
+    vis = np.minimum(cfg.S, (t + 1) // cfg.m)
+    ent = np.minimum(cfg.k, vis) if cfg.kind == "csa" else vis
+    rows = int((ent + np.minimum(cfg.W, t + 1)).sum())
+    return cfg.B * 4.0 * cfg.H * cfg.D * rows
+
+
+def main_stack(args, rank, world, local):
+    """Four prefill layers HCA, HCA, CSA, CSA at T = 262144, 128 heads x dim 128
+    (CSA k = 1024, indexer 4 x 64; HCA ratio 128), independent seeded inputs per
+    layer, all resident in HBM.  value = T / (time of the 4 layers) tokens/s."""
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import build, configs
+    build.build()
+    from long_context_compressed_compress_b200 import inputs, layer
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfgs = configs.STACK.layers
+    if args.impl == "reference":
+        if rank == 0:
+            # the oracle on a row sample of each layer, extrapolated per layer
+            tot = 0.0
+            descr = []
+            for c in cfgs:
+                s = OracleSample(c) if c.kind == "csa" else None
+                if s is None:
+                    import numpy as np
+                    import oracle
+                    x = inputs.layer_inputs(c, device="cpu")
+                    t0 = time.perf_counter()
+                    oracle.hca_layer(x, c.m, c.W, c.tau, c.dtype, rows=[(0, int(r)) for r in
+                                     np.random.default_rng(1234).integers(0, c.T, 4)])
+                    dt = time.perf_counter() - t0
+                    tot += dt / 4 * c.T
+                    descr.append(f"HCA: 4 rows + compression {dt:.1f} s")
+                else:
+                    s.rows(4)
+                    tot += c.T / s.value()
+                    descr.append("CSA: " + s.describe()["sample"])
+            v = cfgs[0].T / tot
+            print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+                              "n_gpus": args.gpus, "steps": 1, "warmup": 0, "higher_is_better": True,
+                              "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                              "config": {"workload": "stack_hhcc_256k"},
+                              "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": os.cpu_count(),
+                                               "kind": "oracle", "sample": "; ".join(descr)},
+                              "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    peaks = load_peaks()
+    xs = [inputs.layer_inputs(c, device="cuda") for c in cfgs]
+    stk = layer.Stack(cfgs, chunk=args.chunk or 16384)
+    stream = torch.cuda.current_stream()
+    ev = {}
+
+    @contextlib.contextmanager
+    def timer(name):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        yield
+        e1.record(stream)
+        ev.setdefault(name, []).append((e0, e1))
+
+    for _ in range(args.warmup):
+        stk.run(xs)
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(local))
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(args.steps):
+        stk.run(xs, timer=timer)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    ms = s0.elapsed_time(s1)
+    if world > 1:
+        ms = max_over_ranks(ms, dev)
+    ms_step = ms / args.steps
+    kern = {k: sum(a.elapsed_time(b) for a, b in v) / args.steps for k, v in ev.items()}
+    flops = {"sparse_attn_fwd": sum(attn_flops(c) for c in cfgs if c.kind == "csa"),
+             "hca_dense_attn_fwd": sum(attn_flops(c) for c in cfgs if c.kind == "hca")}
+    kernels = {}
+    for name, t in kern.items():
+        f = flops.get(name)
+        rate = f / (t * 1e-3) / 1e12 if f else None
+        kernels[name] = {"ms": round(t, 4), "achieved": rate and round(rate, 1), "unit": "TFLOP/s" if f else "",
+                         "frac": rate and round(rate / peaks["bf16_tflops_sustained"], 4)}
+    top = max(flops, key=lambda n: kern.get(n, 0.0))
+    achieved = flops[top] / (kern[top] * 1e-3) / 1e12
+    # end to end: every layer's inputs copied from pinned host memory, the four
+    # layers, the four outputs read back
+    host = [{k: v.cpu().pin_memory() for k, v in x.items()} for x in xs]
+    outs_h = [torch.empty(lay.out.shape, dtype=lay.out.dtype).pin_memory() for lay in stk.layers]
+    h2d = sum(v.numel() * v.element_size() for h in host for v in h.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs_h)
+
+    def e2e_step():
+        for h, x in zip(host, xs):
+            for k, v in h.items():
+                x[k].copy_(v, non_blocking=True)
+        stk.run(xs)
+        for o, lay in zip(outs_h, stk.layers):
+            o.copy_(lay.out, non_blocking=True)
+
+    n_e2e = max(1, min(args.e2e_steps, 3))
+    e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if world > 1:
+        e2e_ms = max_over_ranks(e2e_ms, dev)
+    T = cfgs[0].T
+    line = {
+        "metric": METRIC, "value": job_throughput(world, T, ms_step), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs per layer, drawn on the device)",
+        "config": {"workload": "stack_hhcc_256k", "layers": "HCA,HCA,CSA,CSA", "T": T, "H": cfgs[0].H,
+                   "D": cfgs[0].D, "k": cfgs[2].k, "chunk": stk.layers[2].chunk,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (8.6 GB of q per layer)"},
+        "e2e": {"value": job_throughput(world, T, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": stk.launches * args.steps,
+        "roofline": {"bound": "tensor", "kernel": top, "achieved": achieved,
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel inside a long step)",
+                     "algorithmic_flops_per_step": flops[top]},
+        "kernels": kernels, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 

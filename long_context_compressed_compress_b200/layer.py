@@ -229,3 +229,21 @@ class CsaDecode:
     def replay(self):
         self.graph.replay()
         return self.out
+
+
+class Stack:
+    """An interleaved prefill stack: the layers of ``cfgs`` (e.g. HCA, HCA, CSA,
+    CSA, as in the [attention.hca] interleave_pattern of yfxerp.com/news/211352
+    §3) run one after another, each on its own inputs; the layers do not feed
+    each other (no projections or residual path are part of this layer)."""
+
+    def __init__(self, cfgs, device="cuda", chunk=16384):
+        self.layers = []
+        for c in cfgs:
+            self.layers.append(CsaPrefill(c, device=device, chunk=chunk) if c.kind == "csa"
+                               else HcaPrefill(c, device=device))
+        self.launches = sum(lay.launches for lay in self.layers)
+
+    def run(self, xs, timer=None):
+        """xs: one input dict per layer.  Returns the layers' outputs."""
+        return [lay.run(x, timer=timer) for lay, x in zip(self.layers, xs)]

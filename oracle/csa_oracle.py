@@ -271,19 +271,21 @@ def sparse_attn(q, kv_c, idx, kv_raw, raw_cap, sink, tau, W, positions, rows=Non
     positions [B,T].  ``rows`` optionally restricts the evaluation to a list of
     (b, t) pairs (returned in that order).  Returns float64 out, lse.
     """
-    q, kv_c, kv_raw = _f64(q), _f64(kv_c), _f64(kv_raw)
-    idx = np.asarray(idx)
+    kv_c, kv_raw = _f64(kv_c), _f64(kv_raw)     # q is converted row by row
+    if not isinstance(idx, dict):               # a dict maps (b, t) -> that row's idx
+        idx = np.asarray(idx)
     H = q.shape[2]
     snk = np.full(H, -np.inf) if sink is None else _f64(sink)
     pos = np.asarray(positions)
     pairs = rows if rows is not None else [(b, t) for b in range(q.shape[0]) for t in range(q.shape[1])]
     outs, lses = [], []
     for (b, t) in pairs:
-        sel = idx[b, t][idx[b, t] >= 0]
+        ir = np.asarray(idx[(b, t)])
+        sel = ir[ir >= 0]
         keys = kv_c[b, sel]
         if W > 0:
             keys = np.concatenate([keys, _window_rows(kv_raw[b], raw_cap, int(pos[b, t]), W)], axis=0)
-        o, l = attend_rows(q[b, t], keys, snk, tau)
+        o, l = attend_rows(_f64(q[b, t]), keys, snk, tau)
         outs.append(o)
         lses.append(l)
     return _reshape_rows(outs, lses, q, rows)
@@ -292,7 +294,7 @@ def sparse_attn(q, kv_c, idx, kv_raw, raw_cap, sink, tau, W, positions, rows=Non
 def dense_attn(q, kv_c, kv_raw, raw_cap, sink, tau, W, positions, m, rows=None):
     """HCA attention: each query attends to every visible compressed entry
     ([cf-1] §3.2: no sparse selection, dense attention) plus the raw window and sink."""
-    q, kv_c, kv_raw = _f64(q), _f64(kv_c), _f64(kv_raw)
+    kv_c, kv_raw = _f64(kv_c), _f64(kv_raw)     # q is converted row by row
     H = q.shape[2]
     snk = np.full(H, -np.inf) if sink is None else _f64(sink)
     pos = np.asarray(positions)
@@ -304,7 +306,7 @@ def dense_attn(q, kv_c, kv_raw, raw_cap, sink, tau, W, positions, m, rows=None):
         keys = kv_c[b, :n]
         if W > 0:
             keys = np.concatenate([keys, _window_rows(kv_raw[b], raw_cap, p, W)], axis=0)
-        o, l = attend_rows(q[b, t], keys, snk, tau)
+        o, l = attend_rows(_f64(q[b, t]), keys, snk, tau)
         outs.append(o)
         lses.append(l)
     return _reshape_rows(outs, lses, q, rows)
@@ -361,38 +363,36 @@ def csa_layer(x, m, k, W, tau, dtype, gscale=1.0, rows=None, return_all=False):
     Storage points round once to ``dtype`` ('f32' or 'bf16'); scores to f32 for
     f32 layers and bf16 otherwise.
     """
-    q = _f64(x["q"])
+    q = x["q"]                                  # converted row by row in sparse_attn
     B, T, H, D = q.shape
     pos = np.tile(np.arange(T), (B, 1))
     kv_c = round_out(csa_compress(x["a"], x["b"], x["z"], m), dtype)
     k_src = round_out(csa_compress(x["a_I"], x["b_I"], x["z_I"], m), dtype)
     khat = nvfp4_quantize(k_src, gscale)["xhat"]
-    qhat_all = nvfp4_quantize(_f64(x["q_I"]), gscale)["xhat"]
-    w = _f64(x["w"])
+    w = x["w"]
     if rows is None:
         rows = [(b, t) for b in range(B) for t in range(T)]
     sc_dtype = "f32" if dtype == "f32" else "bf16"
     idx_rows, scores = [], []
     for (b, t) in rows:
-        s = indexer_score(qhat_all[b:b + 1, t:t + 1], khat[b:b + 1], w[b:b + 1, t:t + 1],
-                          pos[b:b + 1, t:t + 1], m)
+        # NVFP4 blocks run along the last dim, so quantising one row is exact
+        qh = nvfp4_quantize(_f64(x["q_I"][b:b + 1, t:t + 1]), gscale)["xhat"]
+        s = indexer_score(qh, khat[b:b + 1], _f64(w[b:b + 1, t:t + 1]), pos[b:b + 1, t:t + 1], m)
         s = round_scores(s, sc_dtype)
         scores.append(s[0, 0])
         idx_rows.append(topk_select(s, pos[b:b + 1, t:t + 1], m, k)[0, 0])
-    idx_full = np.full((B, T, k), -1, dtype=np.int32)
-    for (b, t), ir in zip(rows, idx_rows):
-        idx_full[b, t] = ir
-    out, lse = sparse_attn(q, kv_c, idx_full, x["kv_raw"], T, x["sink"], tau, W, pos, rows=rows)
+    idx_rows_by_bt = {(b, t): ir for (b, t), ir in zip(rows, idx_rows)}
+    out, lse = sparse_attn(q, kv_c, idx_rows_by_bt, x["kv_raw"], T, x["sink"], tau, W, pos, rows=rows)
     res = {"out": round_out(out, dtype), "lse": formats.f32(lse), "idx": np.stack(idx_rows)}
     if return_all:
-        res.update(kv_c=kv_c, k_src=k_src, khat=khat, qhat=qhat_all, score=np.stack(scores))
+        res.update(kv_c=kv_c, k_src=k_src, khat=khat, score=np.stack(scores))
     return res
 
 
 def hca_layer(x, m, W, tau, dtype, rows=None, return_all=False):
     """One HCA layer: 128:1 compression then dense attention over every visible
     entry plus the raw window and sink.  ``rows`` as in ``csa_layer``."""
-    q = _f64(x["q"])
+    q = x["q"]                                  # converted row by row in dense_attn
     B, T, H, D = q.shape
     pos = np.tile(np.arange(T), (B, 1))
     kv_c = round_out(hca_compress(x["a"], x["z"], m), dtype)

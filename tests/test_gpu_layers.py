@@ -65,13 +65,13 @@ def check_csa(L, cfg, rows=None, chunk=None):
     if rows is None:
         rows = [(b, t) for b in range(cfg.B) for t in range(cfg.T)]
     ref = oracle.csa_layer(x, cfg.m, cfg.k, cfg.W, cfg.tau, cfg.dtype, rows=rows, return_all=True)
-    gi = idx_all.cpu().numpy()
+    gi = {(b, t): idx_all[b, t].cpu().numpy() for (b, t) in rows}
     overlaps, near_ok = [], True
     ulp = (lambda v: 2 * formats.bf16(np.abs(v)) * 2.0 ** -8) if cfg.dtype != "f32" else (lambda v: 1e-6 * np.abs(v))
     agree = []
     for n, (b, t) in enumerate(rows):
         ro = set(ref["idx"][n][ref["idx"][n] >= 0].tolist())
-        go = set(gi[b, t][gi[b, t] >= 0].tolist())
+        go = set(gi[(b, t)][gi[(b, t)] >= 0].tolist())
         overlaps.append(1.0 if not ro and not go else len(ro & go) / max(1, len(ro)))
         agree.append(ro == go)
         if ro != go:
@@ -131,6 +131,26 @@ def test_hca_bf16_small_layer(L):
 def test_hca_bf16_h128(L):
     cfg = configs.scaled(configs.STACK.layers[0], T=128 * 24 + 5, seed=13)
     check_hca(L, cfg, sample_rows(cfg.B, cfg.T, 130, 256))
+
+
+def test_hca_bf16_full_size_sampled(L):
+    """HCA prefill at full size: B=2, T=131072, 64 heads, ratio 128."""
+    cfg = configs.HCA_PREFILL
+    check_hca(L, cfg, sample_rows(cfg.B, cfg.T))
+
+
+@pytest.mark.parametrize("layer_no", [0, 1, 2, 3])
+def test_stack_layer_full_size_sampled(L, layer_no):
+    """Each layer of the HCA, HCA, CSA, CSA stack at full size (T=262144, 128
+    heads; CSA k=1024 over 65536 entries, scored in 16384-row chunks as the
+    stack bench runs it), on a row sample."""
+    cfg = configs.STACK.layers[layer_no]
+    rows = sample_rows(cfg.B, cfg.T, 32, 96)
+    if cfg.kind == "csa":
+        check_csa(L, cfg, rows=rows, chunk=16384)
+    else:
+        check_hca(L, cfg, rows)
+    torch.cuda.empty_cache()
 
 
 def test_determinism_and_batch_invariance(L):
