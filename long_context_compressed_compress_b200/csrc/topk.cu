@@ -198,6 +198,221 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const T* __restr
 }
 
 // ---------------------------------------------------------------------------
+// Shared-memory select, one CTA per row, each thread owning a contiguous run.
+// The row's keys are staged so that thread t holds keys [t L, (t+1) L) at
+// shared offset t Lp, with Lp / V odd (V keys per 16-byte vector): the 16-byte
+// reads of a quarter-warp then fall in distinct bank groups.  The first digit's
+// histogram is taken while the row is loaded; each later digit re-reads the
+// runs.  Histogram atomics go to kRunCopies copies picked by lane, so lanes
+// whose keys share a bin (scores crowd into a few exponents) rarely collide.
+// Compaction: per-thread counts of keys > K and == K, two block scans for the
+// output offsets, then every thread writes its own selections in index order.
+// ---------------------------------------------------------------------------
+constexpr int kRunCopies = 8;
+
+template <int NT>
+__device__ __forceinline__ int block_excl_scan_nt(int v, int* wsum, int* total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int inc = warp_incl_scan(v);
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  int before = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int x = wsum[w];
+    before += (w < warp) ? x : 0;
+    tot += x;
+  }
+  __syncthreads();
+  *total = tot;
+  return before + inc - v;
+}
+
+// Run length L (a multiple of V) and padded stride Lp for n keys on NT threads.
+template <int NT, int V>
+__host__ __device__ __forceinline__ void run_shape(int n, int* L, int* Lp) {
+  const int l = ((n + NT - 1) / NT + V - 1) / V * V;
+  *L = l;
+  *Lp = ((l / V) & 1) ? l : l + V;
+}
+
+template <typename T, int NT>
+__global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ score, int T_chunk, int S, int ld,
+                                                      int k, int m, int row0, const int32_t* __restrict__ q_pos0,
+                                                      int32_t* __restrict__ idx) {
+  using KO = KeyOf<T>;
+  using K = typename KO::K;
+  static_assert(sizeof(K) == sizeof(T), "key and score widths match");
+  constexpr int V = 16 / sizeof(K);
+  constexpr int DPT = (256 + NT - 1) / NT;
+  constexpr int top = KO::bits - 8;
+  extern __shared__ __align__(16) uint8_t dsm[];
+  __shared__ int hist[kRunCopies][256];
+  __shared__ int wsum[NT / 32];
+  __shared__ int sel_digit, sel_above;
+
+  const int row = blockIdx.x;
+  const int bi = row / T_chunk;
+  const int r = row - bi * T_chunk;
+  long long nv = (static_cast<long long>(q_pos0[bi]) + row0 + r + 1) / m;
+  if (nv > S) nv = S;
+  if (nv < 0) nv = 0;
+  const int n = static_cast<int>(nv);
+  int32_t* out = idx + static_cast<size_t>(row) * k;
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (n <= k) {
+    for (int i = tid; i < k; i += NT) out[i] = i < n ? i : -1;
+    return;
+  }
+  int L, Lp;
+  run_shape<NT, V>(n, &L, &Lp);
+  K* keys = reinterpret_cast<K*>(dsm);
+  int* hflat = &hist[0][0];
+  const int cp = lane & (kRunCopies - 1);
+  for (int i = tid; i < kRunCopies * 256; i += NT) hflat[i] = 0;
+  __syncthreads();
+
+  // ---- stage the row as keys (16-byte loads where aligned) + first-digit histogram
+  const T* srow = score + static_cast<size_t>(row) * ld;
+  int done = 0;
+  if ((reinterpret_cast<uintptr_t>(srow) & 15) == 0) {
+    const int nvec = n / V;
+#pragma unroll 2
+    for (int g = tid; g < nvec; g += NT) {
+      const uint4 u = reinterpret_cast<const uint4*>(srow)[g];
+      const T* e = reinterpret_cast<const T*>(&u);
+      K kk[V];
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        kk[q] = KO::get(e[q]);
+        atomicAdd(&hist[cp][static_cast<uint32_t>(kk[q]) >> top], 1);
+      }
+      const int i = g * V;
+      const int t = i / L;
+      *reinterpret_cast<uint4*>(keys + static_cast<size_t>(t) * Lp + (i - t * L)) =
+          *reinterpret_cast<const uint4*>(kk);
+    }
+    done = nvec * V;
+  }
+  for (int i = done + tid; i < n; i += NT) {
+    const K key = KO::get(srow[i]);
+    atomicAdd(&hist[cp][static_cast<uint32_t>(key) >> top], 1);
+    const int t = i / L;
+    keys[static_cast<size_t>(t) * Lp + (i - t * L)] = key;
+  }
+  __syncthreads();
+
+  const int cnt = max(0, min(L, n - tid * L));
+  const K* run = keys + static_cast<size_t>(tid) * Lp;
+  uint32_t prefix = 0, pmask = 0;
+  int krem = k;
+#pragma unroll 1
+  for (int shift = top; shift >= 0; shift -= 8) {
+    if (shift != top) {
+      for (int i = tid; i < kRunCopies * 256; i += NT) hflat[i] = 0;
+      __syncthreads();
+      for (int j = 0; j < cnt; j += V) {
+        const uint4 u = *reinterpret_cast<const uint4*>(run + j);
+        const K* kk = reinterpret_cast<const K*>(&u);
+#pragma unroll
+        for (int q = 0; q < V; ++q) {
+          const uint32_t key = kk[q];
+          if (j + q < cnt && (key & pmask) == prefix) atomicAdd(&hist[cp][(key >> shift) & 0xFFu], 1);
+        }
+      }
+      __syncthreads();
+    }
+    // thread t owns digits 255 - DPT t - q (descending), summed over the copies
+    int cq[DPT], csum = 0;
+#pragma unroll
+    for (int q = 0; q < DPT; ++q) {
+      const int d = 255 - DPT * tid - q;
+      int c = 0;
+      if (d >= 0) {
+#pragma unroll
+        for (int c2 = 0; c2 < kRunCopies; ++c2) c += hist[c2][d];
+      }
+      cq[q] = c;
+      csum += c;
+    }
+    int tot;
+    int above = block_excl_scan_nt<NT>(csum, wsum, &tot);
+#pragma unroll
+    for (int q = 0; q < DPT; ++q) {
+      if (above < krem && krem <= above + cq[q]) {
+        sel_digit = 255 - DPT * tid - q;
+        sel_above = above;
+      }
+      above += cq[q];
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(sel_digit) << shift;
+    pmask |= 0xFFu << shift;
+    krem -= sel_above;
+  }
+  // ---- threshold key K = prefix: every key > K, and the first krem keys == K
+  int n_gt = 0, n_eq = 0;
+  for (int j = 0; j < cnt; j += V) {
+    const uint4 u = *reinterpret_cast<const uint4*>(run + j);
+    const K* kk = reinterpret_cast<const K*>(&u);
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      const uint32_t key = kk[q];
+      const bool ok = j + q < cnt;
+      n_gt += ok && key > prefix;
+      n_eq += ok && key == prefix;
+    }
+  }
+  int tot_gt, tot_eq;
+  const int gt_before = block_excl_scan_nt<NT>(n_gt, wsum, &tot_gt);
+  int eq_seen = block_excl_scan_nt<NT>(n_eq, wsum, &tot_eq);
+  int pos = gt_before + min(eq_seen, krem);
+  const int base = tid * L;
+  for (int j = 0; j < cnt; j += V) {
+    const uint4 u = *reinterpret_cast<const uint4*>(run + j);
+    const K* kk = reinterpret_cast<const K*>(&u);
+#pragma unroll
+    for (int q = 0; q < V; ++q) {
+      const uint32_t key = kk[q];
+      if (j + q < cnt) {
+        if (key > prefix) {
+          out[pos++] = base + j + q;
+        } else if (key == prefix) {
+          if (eq_seen < krem) out[pos++] = base + j + q;
+          ++eq_seen;
+        }
+      }
+    }
+  }
+}
+
+template <typename T, int NT>
+size_t run_smem_bytes(int S) {
+  using K = typename KeyOf<T>::K;
+  constexpr int V = 16 / sizeof(K);
+  int L, Lp;
+  run_shape<NT, V>(S, &L, &Lp);
+  return static_cast<size_t>(NT) * (L + V) * sizeof(K);
+}
+
+template <typename T, int NT>
+int launch_topk_run(const T* score, long long rows, int T_chunk, int S, int ld, int k, int m, int row0,
+                    const int32_t* q_pos0, int32_t* idx, cudaStream_t st) {
+  const size_t bytes = run_smem_bytes<T, NT>(S);
+  static int attr = -1;
+  if (attr < static_cast<int>(bytes)) {
+    cudaError_t e = cudaFuncSetAttribute(topk_run_kernel<T, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kTopkSmemMax));
+    if (e != cudaSuccess) return set_cuda_error(e);
+    attr = static_cast<int>(kTopkSmemMax);
+  }
+  topk_run_kernel<T, NT><<<static_cast<unsigned>(rows), NT, bytes, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0,
+                                                                         idx);
+  return check_launch();
+}
+
+// ---------------------------------------------------------------------------
 // Multi-CTA select for a few long BF16 rows (decode: 32 rows of 262144 scores).
 // A row is cut into chunks of kMcChunk keys, one CTA per (row, chunk), and the
 // radix select runs as four launches that meet through a caller workspace:
@@ -452,15 +667,11 @@ int launch_topk(const T* score, int B, int T_chunk, int S, int ld, int k, int m,
   using K = typename KeyOf<T>::K;
   const size_t keys_bytes = static_cast<size_t>(S) * sizeof(K);
   const unsigned grid = static_cast<unsigned>(rows);
-  if (keys_bytes <= kTopkSmemMax) {
-    static int attr = -1;
-    if (attr < static_cast<int>(keys_bytes)) {
-      cudaError_t e = cudaFuncSetAttribute(topk_row_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(kTopkSmemMax));
-      if (e != cudaSuccess) return set_cuda_error(e);
-      attr = static_cast<int>(kTopkSmemMax);
-    }
-    topk_row_kernel<T, true><<<grid, kTopkThreads, keys_bytes, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, idx);
+  (void)keys_bytes;
+  if (S <= 16384 && run_smem_bytes<T, 128>(S) <= kTopkSmemMax) {
+    return launch_topk_run<T, 128>(score, rows, T_chunk, S, ld, k, m, row0, q_pos0, idx, st);
+  } else if (run_smem_bytes<T, 512>(S) <= kTopkSmemMax) {
+    return launch_topk_run<T, 512>(score, rows, T_chunk, S, ld, k, m, row0, q_pos0, idx, st);
   } else {
     topk_row_kernel<T, false><<<grid, kTopkThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, idx);
   }
