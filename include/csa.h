@@ -203,7 +203,8 @@ int topk_select_noalloc(const void* score, int score_dtype, int B, int T_chunk,
  * sink == NULL means sigma = -inf.  W = 0 with sink == NULL gives the
  * compressed branch alone for swa_sink_merge.
  *   q, out [B, T, H, D] (rows row0 .. row0+T_chunk-1 are used), dtype
- *   kv_c [B, kv_bstride, D], idx int32 [B, T_chunk, k], kv_raw [B, raw_cap, D]
+ *   kv_c [B, kv_bstride, D], idx int32 [B, T_chunk, k] (each row: its valid
+ *   entries first, then -1 padding, as topk_select writes it), kv_raw [B, raw_cap, D]
  *   sink fp32 [H] or NULL, lse fp32 [B, T, H] or NULL
  * Requires D in {64, 128}; bf16 runs on tcgen05 (H in {16..128}, H % 16 == 0),
  * fp32 on CUDA cores in fp32.

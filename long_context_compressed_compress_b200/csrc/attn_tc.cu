@@ -76,7 +76,9 @@ struct TcCfg {
   // all-ones A operand (L^T += 1 . P^T) into TMEM; N = 128 keeps them in registers
   static constexpr bool kSumMma = NB == 1;
   static constexpr uint32_t kTmemCols = kSumMma ? 512 : 4 * N;   // S x2, O x2 (+ L x2)
-  static constexpr int kOnesBytes = kSumMma ? kTcTile * 128 : 1024;
+  // all-ones A operand [128 x 16] in the no-swizzle K-major layout (8-row x
+  // 16-byte core matrices, 128 B apart along K, 256 B apart along M)
+  static constexpr int kOnesBytes = kSumMma ? 4096 : 1024;
 };
 
 struct TcUnit {
@@ -258,8 +260,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
   if (warp >= kProd0 && warp < kMmaWarp) {
     // ===================================================================== producer
     const int pw = warp - kProd0;              // producer warp pw: tile rows [RW pw, RW pw + RW)
-    constexpr int RW = kTcTile / C::kProdWarps;
-    constexpr int NI = RW / 32;
+    constexpr int RW = kTcTile / C::kProdWarps;        // 16 or 64 rows per warp
+    constexpr int NI = (RW + 31) / 32;                  // 32-row index chunks per warp
+    const int cbase = (RW * pw) / 32;                   // first 32-row chunk of this warp's rows
     const uint64_t map_q = reinterpret_cast<uint64_t>(&maps.q);
     const uint64_t map_kv = reinterpret_cast<uint64_t>(&maps.kv);
     const uint64_t map_raw = reinterpret_cast<uint64_t>(&maps.raw);
@@ -275,24 +278,31 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       const int plast = p0 + ntok - 1;
       int n_c;
       const int32_t* irow = args.idx + (static_cast<size_t>(b) * args.T_chunk + r0) * args.k;
-      // top-k indices of this lane's rows (RW pw + 32 q + lane) of every entry
-      // tile, loaded up front
+      // top-k indices of tile rows 32 (cbase + q) + lane of every entry tile
+      // (the chunks holding this warp's rows), loaded up front
       int ir[kTcMaxIdxTiles][NI];
       if (args.sparse) {
-        // indices are ascending with -1 padding at the end: binary-search the count
-        int lo = 0, hi = args.k;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (irow[mid] >= 0) lo = mid + 1; else hi = mid;
-        }
-        n_c = lo;
+        // Valid indices form a prefix (-1 pads the end).  Two round trips: lane
+        // l tests the last index of 32-entry chunk l (the number of full chunks
+        // f is a ballot count), then the warp counts chunk f.  This warp's own
+        // tile rows are loaded alongside the first probe.
+        const int Lp = 32 * lane + 31;
+        const int vlast = Lp < args.k ? irow[Lp] : -1;
 #pragma unroll
         for (int i = 0; i < kTcMaxIdxTiles; ++i)
 #pragma unroll
           for (int q = 0; q < NI; ++q) {
-            const int L = i * kTcTile + RW * pw + 32 * q + lane;
-            ir[i][q] = L < n_c ? irow[L] : 0;
+            const int L = i * kTcTile + 32 * (cbase + q) + lane;
+            ir[i][q] = L < args.k ? irow[L] : -1;
           }
+        const int full = __popc(__ballot_sync(0xffffffffu, vlast >= 0));
+        const int Lc = 32 * full + lane;
+        const int vc = Lc < args.k ? irow[Lc] : -1;
+        n_c = 32 * full + __popc(__ballot_sync(0xffffffffu, vc >= 0));
+#pragma unroll
+        for (int i = 0; i < kTcMaxIdxTiles; ++i)
+#pragma unroll
+          for (int q = 0; q < NI; ++q) ir[i][q] = ir[i][q] >= 0 ? ir[i][q] : 0;
       } else {
         n_c = min(args.S, (plast + 1) / args.m);
       }
@@ -354,11 +364,12 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
 #pragma unroll 8
           for (int j = 0; j < RW / 2; ++j) {
             const int rl = 2 * j + half;                   // row within this warp's RW rows
+            const int trow = RW * pw + rl;                  // tile row: chunk trow / 32, lane trow % 32
             int s_g = 0;
 #pragma unroll
             for (int q = 0; q < NI; ++q) {
-              const int v = __shfl_sync(0xffffffffu, tr[q], rl & 31);
-              if ((rl >> 5) == q) s_g = v;
+              const int v = __shfl_sync(0xffffffffu, tr[q], trow & 31);
+              if ((trow >> 5) - cbase == q) s_g = v;
             }
             const int rr = RW * pw + rl;                   // tile row
             const int L = L0 + rr;
@@ -436,8 +447,8 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           if constexpr (C::kSumMma) {
 #pragma unroll
             for (int j = 0; j < kTcTile / 16; ++j)
-              mma_bf16(tmem + 4 * N + ob * N, desc_kmajor(ones_base, 0, j), desc_mnmajor(pbase, kTcTile * 128, j),
-                       idesc_sum, (i > 0 || j > 0) ? 1u : 0u);
+              mma_bf16(tmem + 4 * N + ob * N, make_sdesc(ones_base, 128, 256, kLayoutNone),
+                       desc_mnmajor(pbase, kTcTile * 128, j), idesc_sum, (i > 0 || j > 0) ? 1u : 0u);
           }
           tc_commit(&sm.kv_empty[stage]);
           tc_commit(&sm.p_empty[pb]);
@@ -471,12 +482,24 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       // warpgroup); per-thread row-sum partials unless the MMA keeps the sums
       float mreg[CW];
       float lpart[kSumMma ? 1 : CW];
+      // The running max starts at the head's sink logit: the sink is part of
+      // every denominator, so m >= sigma is a valid stabiliser from the first
+      // row on, and a unit's first tile needs no exact max unless a logit
+      // exceeds its sink by 2^8 (log2 units).  Without a sink, columns start
+      // unset and the first valid rows fix their max exactly.
+      bool allset = true;    // every column of this warpgroup has a running max
 #pragma unroll
-      for (int c = 0; c < CW; ++c) mreg[c] = kNoRowMax;
+      for (int c = 0; c < CW; ++c) {
+        const float sg = sm.sink_l2[(col0 + c) & (args.H - 1)];
+        mreg[c] = sg > -INFINITY ? sg : kNoRowMax;
+        allset = allset && sg > -INFINITY;
+      }
 #pragma unroll
       for (int c = 0; c < (kSumMma ? 1 : CW); ++c) lpart[c] = 0.f;
-      if (row < CW) sm.mcol[wg][row] = kNoRowMax;
-      bool allset = false;   // every column of this warpgroup has a running max
+      if (row < CW) {
+        const float sg = sm.sink_l2[(col0 + row) & (args.H - 1)];
+        sm.mcol[wg][row] = sg > -INFINITY ? sg : kNoRowMax;
+      }
       named_bar_sync(bar_id, 128);
       bool ok = true;
       for (int i = 0; i < inf.nt; ++i, ++gt) {
