@@ -24,7 +24,8 @@ namespace csa {
 
 constexpr int kIdxThreads = 128;
 constexpr int kIdxTilesPerCta = 8;
-constexpr uint32_t kIdxTmemCols = 256;  // acc 128 cols + SFA 4 + SFB 4 (power of two)
+// TMEM columns: accumulator NQ + SFA 4 + SFB 4, rounded to a power of two
+template <int NQ> struct IdxTmem { static constexpr uint32_t cols = NQ == 128 ? 256 : 32; };
 constexpr size_t kIdxSmemFloor = 96 * 1024;  // keeps <= 2 CTAs per SM (TMEM 2 x 256 cols)
 
 struct __align__(128) IdxSmem {
@@ -45,13 +46,18 @@ __device__ __forceinline__ uint32_t cm_off(int r, int c16) { return (r >> 3) * 2
 // 4-byte word r / 32 of that line, byte j = block index along K.
 __device__ __forceinline__ uint32_t sf_off(int r) { return (r & 31) * 16 + (r >> 5) * 4; }
 
-template <int HI, typename TS>
+// NQ = MMA N: 128 (token, head) columns for prefill chunks, 16 for decode
+// (a chunk of at most 16 / HI query tokens): the narrow tile needs 32 TMEM
+// columns and little shared memory, so many CTAs share an SM and keep enough
+// key loads in flight to stream the whole NVFP4 key cache from HBM.
+template <int HI, typename TS, int NQ>
 __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
     const uint8_t* __restrict__ q_fp4, const uint8_t* __restrict__ q_sf, const uint8_t* __restrict__ k_fp4,
     const uint8_t* __restrict__ k_sf, const float* __restrict__ w, float gscale, int T, int row0, int T_chunk,
     int S, int k_bstride, int DI, int m, const int32_t* __restrict__ q_pos0, TS* __restrict__ score, int ld,
     int n_qtiles, int n_chunks, int* __restrict__ status) {
-  constexpr int TQ = 128 / HI;
+  constexpr int TQ = NQ / HI;
+  constexpr uint32_t kIdxTmemCols = IdxTmem<NQ>::cols;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
   IdxSmem& sm = *reinterpret_cast<IdxSmem*>(dsm_raw);
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -87,7 +93,7 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
   {
     const int n = tid;
     const int t = n / HI;
-    const bool ok = t < ntok;
+    const bool ok = n < NQ && t < ntok;
     const size_t qrow = (static_cast<size_t>(bi) * T + row0 + tq0) * HI + n;
     const uint8_t* src = q_fp4 + (ok ? qrow : 0) * dbytes;
     cp_async16(smem_u32(sm.qB + cm_off(n, 0)), src, ok ? 16u : 0u);
@@ -125,8 +131,8 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
-  const uint32_t t_acc = tmem, t_sfa = tmem + 128, t_sfb = tmem + 132;
-  constexpr uint32_t idesc = idesc_nvfp4(128, 128);
+  const uint32_t t_acc = tmem, t_sfa = tmem + NQ, t_sfb = tmem + NQ + 4;
+  constexpr uint32_t idesc = idesc_nvfp4(128, NQ);
   const uint64_t bdesc = make_sdesc(smem_u32(sm.qB), 128, 256, kLayoutNone);
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
 
@@ -153,13 +159,15 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
     // ---- epilogue: this thread owns entry s; columns are (token, head) pairs
     const int s = (et0 + j) * 128 + tid;
     const bool s_ok = s < S;
+    constexpr int CB = NQ < 32 ? NQ : 32;      // columns per TMEM load
 #pragma unroll 1
-    for (int c0 = 0; c0 < 128; c0 += 32) {
-      uint32_t v[32];
-      tmem_ld32(t_acc + lane_base + c0, v);
+    for (int c0 = 0; c0 < NQ; c0 += CB) {
+      uint32_t v[CB];
+      if constexpr (CB == 32) tmem_ld32(t_acc + lane_base + c0, v);
+      else tmem_ld16(t_acc + lane_base + c0, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int tt = 0; tt < 32 / HI; ++tt) {
+      for (int tt = 0; tt < CB / HI; ++tt) {
         const int t = c0 / HI + tt;
         float acc = 0.f;
 #pragma unroll
@@ -194,24 +202,31 @@ extern "C" int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_
   CSA_REQUIRE(HI == 1 || HI == 2 || HI == 4 || HI == 8, CSA_ERR_UNSUPPORTED);
   CSA_REQUIRE(aligned16(q_fp4) && aligned16(k_fp4), CSA_ERR_ALIGNMENT);
   if (B == 0 || T_chunk == 0 || S == 0) return CSA_OK;
-  const int TQ = 128 / HI;
+  const bool narrow = T_chunk * HI <= 16;      // decode-sized chunk: N = 16
+  const int TQ = (narrow ? 16 : 128) / HI;
   const int n_qtiles = (T_chunk + TQ - 1) / TQ;
   const int n_et = (S + 127) / 128;
   const int n_chunks = (n_et + kIdxTilesPerCta - 1) / kIdxTilesPerCta;
   const long long grid = static_cast<long long>(B) * n_qtiles * n_chunks;
   CSA_REQUIRE(grid < (1ll << 31), CSA_ERR_UNSUPPORTED);
-  const size_t smem = sizeof(IdxSmem) + 1024 > kIdxSmemFloor ? sizeof(IdxSmem) + 1024 : kIdxSmemFloor;
+  const size_t smem_min = sizeof(IdxSmem) + 1024;
+  const size_t smem = narrow ? smem_min : (smem_min > kIdxSmemFloor ? smem_min : kIdxSmemFloor);
   const float g = q_gscale * k_gscale;
   int* status = device_status_ptr();
   CSA_REQUIRE(status != nullptr, CSA_ERR_CUDA);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-#define CSA_IDX_LAUNCH(HIV, TS)                                                                                \
+#define CSA_IDX_LAUNCH_NQ(HIV, TS, NQV)                                                                        \
   do {                                                                                                         \
-    cudaFuncSetAttribute(indexer_kernel<HIV, TS>, cudaFuncAttributeMaxDynamicSharedMemorySize,                 \
+    cudaFuncSetAttribute(indexer_kernel<HIV, TS, NQV>, cudaFuncAttributeMaxDynamicSharedMemorySize,            \
                          static_cast<int>(smem));                                                              \
-    indexer_kernel<HIV, TS><<<static_cast<unsigned>(grid), kIdxThreads, smem, st>>>(                           \
+    indexer_kernel<HIV, TS, NQV><<<static_cast<unsigned>(grid), kIdxThreads, smem, st>>>(                      \
         q_fp4, q_sf, k_fp4, k_sf, w, g, T, row0, T_chunk, S, k_bstride, DI, m, q_pos0, static_cast<TS*>(score), \
         score_ld, n_qtiles, n_chunks, status);                                                                 \
+  } while (0)
+#define CSA_IDX_LAUNCH(HIV, TS)                                 \
+  do {                                                          \
+    if (narrow) CSA_IDX_LAUNCH_NQ(HIV, TS, 16);                 \
+    else CSA_IDX_LAUNCH_NQ(HIV, TS, 128);                       \
   } while (0)
 #define CSA_IDX_DT(HIV)                                                \
   do {                                                                 \
@@ -226,5 +241,6 @@ extern "C" int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_
   }
 #undef CSA_IDX_DT
 #undef CSA_IDX_LAUNCH
+#undef CSA_IDX_LAUNCH_NQ
   return check_launch();
 }

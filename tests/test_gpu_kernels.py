@@ -207,6 +207,35 @@ def test_indexer_score_row_chunks(ops):
         torch.testing.assert_close(part, full[:, r0:r0 + tc], rtol=0, atol=0)
 
 
+@pytest.mark.parametrize("HI", [2, 4, 8])
+def test_indexer_score_decode_chunks(ops, HI):
+    """Chunks of 1..16/HI query rows take the narrow (N = 16) tile: each chunk
+    matches the oracle, with long key rows spanning many entry tiles."""
+    B, T, m, DI = 3, 12, 4, 64
+    S = 1500
+    qi, ki, q4, qs, k4, ks = _quant_inputs(ops, B, T, S, HI, DI, 41)
+    w = torch.rand((B, T, HI), generator=torch.Generator().manual_seed(7))
+    pos0 = torch.tensor([4 * S - 12, 4 * 700, 4 * S + 40], dtype=torch.int32)
+    qhat = oracle.nvfp4_quantize(qi)["xhat"]
+    khat = oracle.nvfp4_quantize(ki)["xhat"]
+    pos = np.arange(T)[None] + pos0.numpy()[:, None]
+    ref = oracle.indexer_score(qhat, khat, w, pos, m)
+    wd, pd = w.cuda(), pos0.cuda()
+    r0 = 0
+    for tc in (1, 16 // HI, 1, max(1, 8 // HI), T):
+        tc = min(tc, T - r0)
+        if tc <= 0:
+            break
+        part = torch.full((B, tc, S), float("nan"), dtype=torch.float32, device="cuda")
+        ops.indexer_score(q4, qs, k4, ks, wd, pd, part, S, m, row0=r0, T_chunk=tc)
+        got = _np(part)
+        rr = ref[:, r0:r0 + tc]
+        vis = ~np.isnan(rr)
+        np.testing.assert_allclose(got[vis], rr[vis], rtol=2e-6, atol=1e-6)
+        assert np.all(np.isnan(got[~vis]))
+        r0 += tc
+
+
 # ------------------------------------------------------------------ top-k
 
 @pytest.mark.parametrize("sdt", ["f32", "bf16"])
