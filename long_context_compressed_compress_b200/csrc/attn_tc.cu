@@ -82,7 +82,7 @@ struct TcCfg {
 };
 
 struct TcUnit {
-  int b, r0, ntok, n_c, n_w, jlo, p0, nt;
+  int b, r0, ntok, n_c, n_w, jlo, p0, nt, hoff;
   int n_all;   // leading rows valid for every token of the unit
   int n_cp;    // n_c rounded up to 4: window rows start here
 };
@@ -130,6 +130,8 @@ struct TcArgs {
   int hshift;            // log2(H)
   int sparse;            // 1: CSA (idx), 0: HCA (all visible entries)
   int units_per_b;
+  int Hq;                // heads per token in q / out / lse / sink (H = heads per unit)
+  int hsplit;            // units per token (Hq / H): few-token calls split the heads
   int n_units;
   int kv_rows, raw_rows; // rows of the kv / raw tensor maps (an index equal to them is out of range)
 };
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     fence_mbar_init();
   }
   for (int h = threadIdx.x; h < 128; h += blockDim.x)
-    sm.sink_l2[h] = (args.sink != nullptr && h < args.H) ? args.sink[h] * 1.4426950408889634f : -INFINITY;
+    sm.sink_l2[h] = (args.sink != nullptr && h < args.Hq) ? args.sink[h] * 1.4426950408889634f : -INFINITY;
   for (int o = threadIdx.x * 16; o < C::kOnesBytes; o += blockDim.x * 16)
     *reinterpret_cast<uint4*>(sm.ones + o) = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
   fence_proxy_async();
@@ -272,7 +274,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       const int slot = it & 1;
       if (it >= 2 && !tc_wait(&sm.q_empty[slot], ((it >> 1) - 1) & 1, args.status, abort_flag)) break;
       const int b = u / args.units_per_b;
-      const int r0 = (u - b * args.units_per_b) * args.G;
+      const int ul = u - b * args.units_per_b;
+      const int r0 = (ul / args.hsplit) * args.G;
+      const int hoff = (ul % args.hsplit) * args.H;
       const int ntok = min(args.G, args.T_chunk - r0);
       const int p0 = args.q_pos0[b] + args.row0 + r0;
       const int plast = p0 + ntok - 1;
@@ -316,15 +320,15 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       const int nt = max(1, (n_rows + kTcTile - 1) / kTcTile);
       const int n_all = args.G > 1 ? min(n_c, (p0 + 1) / args.m) : (n_c == n_cp ? n_rows : n_c);
       if (pw == 0 && lane == 0) {
-        sm.info[slot] = TcUnit{b, r0, ntok, n_c, n_w, jlo, p0, nt, n_all, n_cp};
+        sm.info[slot] = TcUnit{b, r0, ntok, n_c, n_w, jlo, p0, nt, hoff, n_all, n_cp};
         // ---- Q: per token one box of H rows (token-major, head-minor) per
         // 64-column half; only the unit's ntok tokens, so no box leaves q
-        const int qrow0 = (b * args.Tq + args.row0 + r0) * args.H;
+        const int qrow0 = (b * args.Tq + args.row0 + r0) * args.Hq + hoff;
         mbar_arrive_expect_tx(&sm.q_full[slot], ntok * args.H * kTcDim * 2);
         for (int g = 0; g < ntok; ++g) {
           const uint32_t qd = smem_u32(sm.q[slot]) + g * args.H * 128;
-          tma_load_2d(qd, map_q, 0, qrow0 + g * args.H, &sm.q_full[slot]);
-          tma_load_2d(qd + N * 128, map_q, 64, qrow0 + g * args.H, &sm.q_full[slot]);
+          tma_load_2d(qd, map_q, 0, qrow0 + g * args.Hq, &sm.q_full[slot]);
+          tma_load_2d(qd + N * 128, map_q, 64, qrow0 + g * args.Hq, &sm.q_full[slot]);
         }
       }
       // ---- KV tiles
@@ -490,14 +494,14 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       bool allset = true;    // every column of this warpgroup has a running max
 #pragma unroll
       for (int c = 0; c < CW; ++c) {
-        const float sg = sm.sink_l2[(col0 + c) & (args.H - 1)];
+        const float sg = sm.sink_l2[inf.hoff + ((col0 + c) & (args.H - 1))];
         mreg[c] = sg > -INFINITY ? sg : kNoRowMax;
         allset = allset && sg > -INFINITY;
       }
 #pragma unroll
       for (int c = 0; c < (kSumMma ? 1 : CW); ++c) lpart[c] = 0.f;
       if (row < CW) {
-        const float sg = sm.sink_l2[(col0 + row) & (args.H - 1)];
+        const float sg = sm.sink_l2[inf.hoff + ((col0 + row) & (args.H - 1))];
         sm.mcol[wg][row] = sg > -INFINITY ? sg : kNoRowMax;
       }
       named_bar_sync(bar_id, 128);
@@ -705,7 +709,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         }
         const float mcl = mreg[0] * 0.f + sm.mcol[wg][c];
         const int col = col0 + c;
-        const int h = col & (args.H - 1);
+        const int h = inf.hoff + (col & (args.H - 1));
         float scale = 0.f, lse_v = -INFINITY;
         if (mcl > 0.5f * kNoRowMax) {
           const float sg = sm.sink_l2[h];
@@ -718,7 +722,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         if (lane < CW) sm.alpha[wg][c] = scale;
         const int g = col >> args.hshift;
         if (args.lse != nullptr && lane < CW && g < inf.ntok)
-          args.lse[(static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + g) * args.H + h] = lse_v;
+          args.lse[(static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + g) * args.Hq + h] = lse_v;
       }
       named_bar_sync(bar_id, 128);
       if (threadIdx.x == 0) CSA_TR(it, 14, 1);
@@ -730,7 +734,8 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         if constexpr (CW == 32) tmem_ld16(oaddr + 16, v + 16);
         tmem_ld_wait();
         if (threadIdx.x == 0) CSA_TR(it, 14, 2);
-        __nv_bfloat16* obase = args.out + (static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0) * args.H * kTcDim + d;
+        __nv_bfloat16* obase =
+            args.out + ((static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0) * args.Hq + inf.hoff) * kTcDim + d;
 #pragma unroll
         for (int c = 0; c < CW; ++c) {
           const int col = col0 + c;
@@ -811,6 +816,15 @@ int launch_attn_tc(const void* q, const void* kv_c, const int32_t* idx, const vo
     CSA_REQUIRE(H == 16 || H == 32 || H == 64 || H == 128, CSA_ERR_UNSUPPORTED);
     G = 128 / H;
   }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Few query rows (decode): split 128 heads into two 64-head units, which
+  // doubles the CTAs at work and uses the N = 64 tile; the extra gather of the
+  // same KV rows is small when there are few rows.
+  const int Hq = H;
+  const int hsplit = (sparse && H == 128 && static_cast<long long>(B) * T_chunk < sms) ? 2 : 1;
+  H = Hq / hsplit;
   const int N = G * H;
   TcArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -829,13 +843,15 @@ int launch_attn_tc(const void* q, const void* kv_c, const int32_t* idx, const vo
   a.G = G;
   a.hshift = 31 - __builtin_clz(static_cast<unsigned>(H));
   a.sparse = sparse;
-  a.units_per_b = (T_chunk + G - 1) / G;
+  a.Hq = Hq;
+  a.hsplit = hsplit;
+  a.units_per_b = (T_chunk + G - 1) / G * hsplit;
   const long long nu = static_cast<long long>(B) * a.units_per_b;
   CSA_REQUIRE(nu < (1ll << 31), CSA_ERR_UNSUPPORTED);
   a.n_units = static_cast<int>(nu);
   if (a.n_units == 0) return CSA_OK;
   if (sparse) CSA_REQUIRE(k <= kTcMaxIdxTiles * kTcTile, CSA_ERR_UNSUPPORTED);
-  const long long q_rows = static_cast<long long>(B) * Tq * H;
+  const long long q_rows = static_cast<long long>(B) * Tq * Hq;
   const long long kv_rows = static_cast<long long>(B) * kv_bstride;
   const long long raw_rows = static_cast<long long>(B) * a.raw_cap;
   CSA_REQUIRE(q_rows < (1ll << 31) && kv_rows < (1ll << 31) - 1 && raw_rows < (1ll << 31) - 1, CSA_ERR_UNSUPPORTED);

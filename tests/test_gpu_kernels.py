@@ -335,6 +335,33 @@ def test_sparse_attn(ops, dtype, H, D, k):
                                atol=1e-4 if dtype == "f32" else 2.0 ** -8)
 
 
+def test_sparse_attn_few_rows_head_split(ops):
+    """A call with fewer query rows than SMs and 128 heads runs each row as two
+    64-head units: a row chunk [1200, 1240) of two sequences vs the oracle,
+    including lse, with rows outside the chunk left untouched."""
+    B, T, m, W, H, D, k = 2, 1300, 4, 128, 128, 128, 300
+    S = T // m
+    tau = 1.0 / np.sqrt(D)
+    q, kv_c, raw, sink = _attn_inputs(B, T, H, D, S, "bf16", 31)
+    pos0 = torch.tensor([0, 7], dtype=torch.int32)
+    pos = np.arange(T)[None] + pos0.numpy()[:, None]
+    r0, tc = 1200, 40
+    idx_full = oracle.topk_select(np.random.default_rng(2).standard_normal((B, T, S)), pos, m, k)
+    idx_chunk = torch.from_numpy(np.ascontiguousarray(idx_full[:, r0:r0 + tc]))
+    out = torch.zeros((B, T, H, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((B, T, H), dtype=torch.float32, device="cuda")
+    ops.sparse_attn_fwd(q.cuda(), kv_c.cuda(), idx_chunk.cuda(), raw.cuda(), sink.cuda(), tau, W, pos0.cuda(), out,
+                        lse, row0=r0, T_chunk=tc)
+    rows = [(b, t) for b in range(B) for t in range(r0, r0 + tc)]
+    ro, rl = oracle.sparse_attn(q, kv_c, {(b, t): idx_full[b, t] for (b, t) in rows}, raw, T, sink, tau, W, pos,
+                                rows=rows)
+    got = np.stack([_np(out[b, t]) for (b, t) in rows])
+    _attn_tol("bf16")(got, oracle.round_out(ro, "bf16"))
+    gl = np.stack([lse[b, t].cpu().numpy() for (b, t) in rows])
+    np.testing.assert_allclose(gl, rl, rtol=0, atol=2.0 ** -8)
+    assert float(out[:, :r0].abs().max()) == 0.0 and float(out[:, r0 + tc:].abs().max()) == 0.0
+
+
 @pytest.mark.parametrize("dtype,H,D,m", [("f32", 8, 64, 4), ("bf16", 64, 128, 16), ("bf16", 128, 128, 32),
                                          ("bf16", 16, 128, 4), ("bf16", 32, 128, 128), ("bf16", 64, 128, 128)])
 def test_hca_dense_attn(ops, dtype, H, D, m):
