@@ -138,7 +138,9 @@ int nvfp4_quantize(const void* x, int in_dtype, int64_t rows, int D, float gscal
  *   k_fp4 [B, k_bstride, DI/2], k_sf [B, k_bstride, DI/16], entries s < S used
  *   score [B, T_chunk, score_ld] in score_dtype, rows r in [0, T_chunk) at
  *   positions q_pos0[b] + row0 + r.  Only visible (r, s) pairs are written.
- * Requires DI in {32, 64}, HI in {1, 2, 4, 8}, score_ld >= S.
+ * Requires DI in {32, 64}, HI in {1, 2, 4, 8}, score_ld >= S; q_fp4 and k_fp4
+ * 16-byte aligned, and k_sf 4-byte aligned when DI = 64 (else
+ * CSA_ERR_ALIGNMENT).
  */
 int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_gscale,
                   const uint8_t* k_fp4, const uint8_t* k_sf, float k_gscale,

@@ -23,15 +23,21 @@
 namespace csa {
 
 constexpr int kIdxThreads = 128;
-constexpr int kIdxTilesPerCta = 8;
+// entry tiles per CTA and shared-memory stages: the narrow (decode) tile
+// streams more tiles per CTA through a deeper ring
+template <int NQ> struct IdxShape {
+  static constexpr int tiles = NQ == 128 ? 8 : 16;
+  static constexpr int stages = NQ == 128 ? 2 : 4;
+};
 // TMEM columns: accumulator NQ + SFA 4 + SFB 4, rounded to a power of two
 template <int NQ> struct IdxTmem { static constexpr uint32_t cols = NQ == 128 ? 256 : 32; };
 constexpr size_t kIdxSmemFloor = 96 * 1024;  // keeps <= 2 CTAs per SM (TMEM 2 x 256 cols)
 
+template <int NS>
 struct __align__(128) IdxSmem {
   uint8_t qB[128 * 32];
-  uint8_t kA[2][128 * 32];
-  uint8_t sfa[2][512];
+  uint8_t kA[NS][128 * 32];
+  uint8_t sfa[NS][512];
   uint8_t sfb[512];
   float w[128];
   uint64_t mbar;
@@ -59,7 +65,9 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
   constexpr int TQ = NQ / HI;
   constexpr uint32_t kIdxTmemCols = IdxTmem<NQ>::cols;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
-  IdxSmem& sm = *reinterpret_cast<IdxSmem*>(dsm_raw);
+  constexpr int NS = IdxShape<NQ>::stages;
+  constexpr int kTilesPerCta = IdxShape<NQ>::tiles;
+  IdxSmem<NS>& sm = *reinterpret_cast<IdxSmem<NS>*>(dsm_raw);
   const int tid = threadIdx.x, warp = tid >> 5;
 
   int blk = blockIdx.x;
@@ -72,8 +80,8 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
   long long vis_last = (pbase + ntok - 1 + 1) / m;
   if (vis_last > S) vis_last = S;
   const int n_et = static_cast<int>((vis_last + 127) / 128);
-  const int et0 = ch * kIdxTilesPerCta;
-  const int et1 = min(n_et, et0 + kIdxTilesPerCta);
+  const int et0 = ch * kTilesPerCta;
+  const int et1 = min(n_et, et0 + kTilesPerCta);
   if (et0 >= et1) return;  // uniform: nothing visible for this CTA
   const int ntiles = et1 - et0;
 
@@ -115,17 +123,23 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
     cp_async16(smem_u32(sm.kA[stage] + cm_off(r, 0)), src, ok ? 16u : 0u);
     cp_async16(smem_u32(sm.kA[stage] + cm_off(r, 1)), src + (dbytes > 16 ? 16 : 0),
                (ok && dbytes > 16) ? 16u : 0u);
-    uint32_t sfw = 0;
-    if (ok) {
-      const uint8_t* sp = k_sf + krow * sfn;
-      for (int j = 0; j < sfn; ++j) sfw |= static_cast<uint32_t>(sp[j]) << (8 * j);
+    if (sfn == 4) {
+      // the row's four scale bytes as one asynchronous 4-byte copy
+      cp_async4(smem_u32(sm.sfa[stage] + sf_off(r)), k_sf + krow * 4, ok ? 4u : 0u);
+    } else {
+      uint32_t sfw = 0;
+      if (ok) {
+        const uint8_t* sp = k_sf + krow * sfn;
+        for (int j = 0; j < sfn; ++j) sfw |= static_cast<uint32_t>(sp[j]) << (8 * j);
+      }
+      *reinterpret_cast<uint32_t*>(sm.sfa[stage] + sf_off(r)) = sfw;
     }
-    *reinterpret_cast<uint32_t*>(sm.sfa[stage] + sf_off(r)) = sfw;
   };
-  load_k_tile(et0, 0);
-  cp_async_commit();
-  if (ntiles > 1) load_k_tile(et0 + 1, 1);
-  cp_async_commit();
+#pragma unroll
+  for (int p = 0; p < NS; ++p) {
+    if (p < ntiles) load_k_tile(et0 + p, p);
+    cp_async_commit();
+  }
 
   tc_fence_before();
   __syncthreads();
@@ -137,8 +151,8 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
 
   for (int j = 0; j < ntiles; ++j) {
-    const int stage = j & 1;
-    cp_async_wait<1>();
+    const int stage = j % NS;
+    cp_async_wait<NS - 1>();
     fence_proxy_async();
     __syncthreads();
     if (sm.abort_flag) break;
@@ -152,8 +166,8 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
     }
     if (!mbar_wait(&sm.mbar, static_cast<uint32_t>(j & 1), status)) sm.abort_flag = 1;
     tc_fence_after();
-    // the MMA has consumed this stage: prefetch two tiles ahead into it
-    if (j + 2 < ntiles) load_k_tile(et0 + j + 2, stage);
+    // the MMA has consumed this stage: prefetch NS tiles ahead into it
+    if (j + NS < ntiles) load_k_tile(et0 + j + NS, stage);
     cp_async_commit();
 
     // ---- epilogue: this thread owns entry s; columns are (token, head) pairs
@@ -201,15 +215,17 @@ extern "C" int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_
   CSA_REQUIRE(DI == 32 || DI == 64, CSA_ERR_UNSUPPORTED);
   CSA_REQUIRE(HI == 1 || HI == 2 || HI == 4 || HI == 8, CSA_ERR_UNSUPPORTED);
   CSA_REQUIRE(aligned16(q_fp4) && aligned16(k_fp4), CSA_ERR_ALIGNMENT);
+  CSA_REQUIRE(DI != 64 || (reinterpret_cast<uintptr_t>(k_sf) & 3) == 0, CSA_ERR_ALIGNMENT);
   if (B == 0 || T_chunk == 0 || S == 0) return CSA_OK;
   const bool narrow = T_chunk * HI <= 16;      // decode-sized chunk: N = 16
   const int TQ = (narrow ? 16 : 128) / HI;
   const int n_qtiles = (T_chunk + TQ - 1) / TQ;
   const int n_et = (S + 127) / 128;
-  const int n_chunks = (n_et + kIdxTilesPerCta - 1) / kIdxTilesPerCta;
+  const int tiles_per_cta = narrow ? IdxShape<16>::tiles : IdxShape<128>::tiles;
+  const int n_chunks = (n_et + tiles_per_cta - 1) / tiles_per_cta;
   const long long grid = static_cast<long long>(B) * n_qtiles * n_chunks;
   CSA_REQUIRE(grid < (1ll << 31), CSA_ERR_UNSUPPORTED);
-  const size_t smem_min = sizeof(IdxSmem) + 1024;
+  const size_t smem_min = (narrow ? sizeof(IdxSmem<IdxShape<16>::stages>) : sizeof(IdxSmem<IdxShape<128>::stages>)) + 1024;
   const size_t smem = narrow ? smem_min : (smem_min > kIdxSmemFloor ? smem_min : kIdxSmemFloor);
   const float g = q_gscale * k_gscale;
   int* status = device_status_ptr();
