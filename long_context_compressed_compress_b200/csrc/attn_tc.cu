@@ -75,7 +75,13 @@ struct TcCfg {
   // N = 64: the per-column row sums come from a second PV-shaped MMA with an
   // all-ones A operand (L^T += 1 . P^T) into TMEM; N = 128 keeps them in registers
   static constexpr bool kSumMma = NB == 1;
-  static constexpr uint32_t kTmemCols = kSumMma ? 512 : 4 * N;   // S x2, O x2 (+ L x2)
+  // S^T and P^T buffers: three for N = 64, so QK runs two tiles ahead of the
+  // softmax and ahead of the PV of the tile before (the tensor pipe executes in
+  // issue order); two for N = 128 (TMEM is full)
+  static constexpr int kSBuf = NB == 1 ? 3 : 2;
+  static constexpr uint32_t kOCol = kSBuf * N;             // O^T x2 after the S buffers
+  static constexpr uint32_t kLCol = (kSBuf + 2) * N;       // L^T x2 (row-sum MMA)
+  static constexpr uint32_t kTmemCols = 512;               // 448 or 512 used
   // all-ones A operand [128 x 16] in the no-swizzle K-major layout (8-row x
   // 16-byte core matrices, 128 B apart along K, 256 B apart along M)
   static constexpr int kOnesBytes = kSumMma ? 4096 : 1024;
@@ -100,15 +106,17 @@ struct __align__(1024) TcSmem {
   using C = TcCfg<NB>;
   uint8_t q[2][C::kQBytes];
   uint8_t kv[C::kStages][C::kKVBytes];
-  uint8_t p[2][C::kPBytes];
+  uint8_t p[C::kSBuf][C::kPBytes];
   uint8_t ones[C::kOnesBytes];   // bf16 1.0 (A operand of the row-sum MMA)
   uint64_t kv_full[C::kStages], kv_empty[C::kStages];
-  uint64_t q_full[2], q_empty[2], s_full[2], s_free[2], p_full[2], p_empty[2], o_full[2], o_empty[2];
+  uint64_t q_full[2], q_empty[2], o_full[2], o_empty[2];
+  uint64_t s_full[C::kSBuf], s_free[C::kSBuf], p_full[C::kSBuf], p_empty[C::kSBuf];
   float xch[C::kGroups][4][C::kCW];
   float mcol[C::kGroups][C::kCW];
   float alpha[C::kGroups][C::kCW];
   float dlt[C::kGroups][C::kCW];
   float sink_l2[128];      // sink logits in log2 units (-inf without a sink)
+  int taint[2];            // unit sequence number + 1 when a unit must be recomputed exactly
   TcUnit info[2];
   uint32_t tmem;
   int abort_flag;
@@ -182,6 +190,9 @@ __device__ __forceinline__ void fadd2(float& x0, float& x1, float y0, float y1) 
 // Running-max sentinel for a column that has seen no valid row yet (finite, so
 // every softmax argument stays finite; masked rows are -inf and give 0).
 constexpr float kNoRowMax = -1e30f;
+// Largest softmax argument (log2 units above the running max) taken without a
+// group-wide max update; larger ones mark the unit for exact recomputation.
+constexpr float kClampD = 64.0f;
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -215,6 +226,74 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
   return (c >> 3) * (rows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
 }
 
+// Exact fallback for one unit, on CUDA cores: every (token, head) column of
+// the unit by one warp at a time (lane = 4 head dims), an online softmax in
+// fp32 over the entries and window rows, then the sink, as the formula states.
+// Used only for units whose fast path was inexact (a logit above the seeded
+// max by more than 2^64, or every weight underflowing).
+__device__ __noinline__ void tc_unit_exact(const TcArgs a, const TcUnit inf, const float* sink_l2, int n_cols,
+                                           int nwarps) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int col = warp; col < n_cols; col += nwarps) {
+    const int g = col >> a.hshift;
+    if (g >= inf.ntok) continue;
+    const int h = inf.hoff + (col & (a.H - 1));
+    const int p = inf.p0 + g;
+    const size_t qrow = (static_cast<size_t>(inf.b) * a.Tq + a.row0 + inf.r0 + g) * a.Hq + h;
+    float qv[4];
+    {
+      const uint2 u = *reinterpret_cast<const uint2*>(a.q + qrow * kTcDim + 4 * lane);
+      const __nv_bfloat162 q01 = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+      const __nv_bfloat162 q23 = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+      qv[0] = __low2float(q01); qv[1] = __high2float(q01); qv[2] = __low2float(q23); qv[3] = __high2float(q23);
+    }
+    float m = -INFINITY, l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    auto visit = [&](const __nv_bfloat16* row) {
+      const uint2 u = *reinterpret_cast<const uint2*>(row + 4 * lane);
+      const __nv_bfloat162 k01 = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+      const __nv_bfloat162 k23 = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+      const float kv[4] = {__low2float(k01), __high2float(k01), __low2float(k23), __high2float(k23)};
+      float dot = qv[0] * kv[0] + qv[1] * kv[1] + qv[2] * kv[2] + qv[3] * kv[3];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      const float x = dot * a.scale_log2;
+      const float mn = fmaxf(m, x);
+      const float corr = exp2f(m - mn);
+      const float pw = exp2f(x - mn);
+      l = fmaf(l, corr, pw);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] = fmaf(acc[e], corr, pw * kv[e]);
+      m = mn;
+    };
+    if (a.sparse) {
+      const int32_t* ir = a.idx + (static_cast<size_t>(inf.b) * a.T_chunk + inf.r0 + g) * a.k;
+      for (int j = 0; j < inf.n_c; ++j)
+        visit(a.kv_c + (static_cast<size_t>(inf.b) * a.kv_bstride + ir[j]) * kTcDim);
+    } else {
+      const int nv = min(a.S, (p + 1) / a.m);
+      for (int e = 0; e < nv; ++e) visit(a.kv_c + (static_cast<size_t>(inf.b) * a.kv_bstride + e) * kTcDim);
+    }
+    if (a.W > 0)
+      for (int j = max(0, p - a.W + 1); j <= p; ++j)
+        visit(a.kv_raw + (static_cast<size_t>(inf.b) * a.raw_cap + (j % a.raw_cap)) * kTcDim);
+    float scale = 0.f, lse_v = -INFINITY;
+    if (l > 0.f) {
+      const float sg = sink_l2[h];
+      const float mx = fmaxf(m, sg);
+      const float f = exp2f(m - mx);
+      scale = __fdiv_rn(f, fmaf(l, f, exp2f(sg - mx)));
+      lse_v = (m + log2f(l)) * 0.6931471805599453f;
+    }
+    const __nv_bfloat162 o01 = __floats2bfloat162_rn(acc[0] * scale, acc[1] * scale);
+    const __nv_bfloat162 o23 = __floats2bfloat162_rn(acc[2] * scale, acc[3] * scale);
+    uint2 ov;
+    ov.x = *reinterpret_cast<const uint32_t*>(&o01);
+    ov.y = *reinterpret_cast<const uint32_t*>(&o23);
+    *reinterpret_cast<uint2*>(a.out + qrow * kTcDim + 4 * lane) = ov;
+    if (a.lse != nullptr && lane == 0) a.lse[qrow] = lse_v;
+  }
+}
+
 template <int NB>
 __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const TcArgs args, const __grid_constant__ TcMaps maps) {
   using C = TcCfg<NB>;
@@ -235,14 +314,18 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.q_full[s], 1);
       mbar_init(&sm.q_empty[s], 1 + 128 * C::kGroups);
+      mbar_init(&sm.o_full[s], 1);
+      mbar_init(&sm.o_empty[s], 128 * C::kGroups);
+    }
+    for (int s = 0; s < C::kSBuf; ++s) {
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.s_free[s], 128 * C::kGroups);
       mbar_init(&sm.p_full[s], 128 * C::kGroups);
       mbar_init(&sm.p_empty[s], 1);
-      mbar_init(&sm.o_full[s], 1);
-      mbar_init(&sm.o_empty[s], 128 * C::kGroups);
     }
     sm.abort_flag = 0;
+    sm.taint[0] = 0;
+    sm.taint[1] = 0;
     fence_mbar_init();
   }
   for (int h = threadIdx.x; h < 128; h += blockDim.x)
@@ -264,6 +347,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     const int pw = warp - kProd0;              // producer warp pw: tile rows [RW pw, RW pw + RW)
     constexpr int RW = kTcTile / C::kProdWarps;        // 16 or 64 rows per warp
     constexpr int NI = (RW + 31) / 32;                  // 32-row index chunks per warp
+    static_assert(RW % 32 == 0, "each producer warp owns whole 32-row index chunks");
     const int cbase = (RW * pw) / 32;                   // first 32-row chunk of this warp's rows
     const uint64_t map_q = reinterpret_cast<uint64_t>(&maps.q);
     const uint64_t map_kv = reinterpret_cast<uint64_t>(&maps.kv);
@@ -353,6 +437,31 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           } else {
             mbar_arrive(&sm.kv_full[stage]);
           }
+        } else if (args.sparse && L0 + kTcTile <= n_c) {
+          // every row of the tile is a selected entry: lean issue loop (row base
+          // pointer hoisted, one shuffle per row pair, swizzle term constant
+          // after unrolling: tile row RW pw + 2 j + half has (row & 7) =
+          // (2 j & 7) | half because RW pw is a multiple of 32)
+          int tr[NI];
+#pragma unroll
+          for (int q = 0; q < NI; ++q) tr[q] = 0;
+#pragma unroll
+          for (int ii = 0; ii < kTcMaxIdxTiles; ++ii)
+            if (ii == i) {
+#pragma unroll
+              for (int q = 0; q < NI; ++q) tr[q] = ir[ii][q];
+            }
+          const int half = lane >> 4, c = lane & 15;
+          const __nv_bfloat16* rb = args.kv_c + static_cast<size_t>(b) * args.kv_bstride * kTcDim + c * 8;
+          const uint32_t dbase = ks + (c >> 3) * (kTcTile * 128) + (RW * pw + half) * 128;
+          const uint32_t cx = static_cast<uint32_t>((c & 7) ^ half);
+#pragma unroll
+          for (int j = 0; j < RW / 2; ++j) {
+            const int s_g = __shfl_sync(0xffffffffu, tr[(2 * j) >> 5], (2 * j + half) & 31);
+            const uint32_t dst = dbase + j * 256 + ((cx ^ static_cast<uint32_t>((2 * j) & 7)) << 4);
+            cp_async16(dst, rb + static_cast<size_t>(s_g) * kTcDim, 16u);
+          }
+          cp_async_mbar_arrive(&sm.kv_full[stage]);
         } else {
           // gather: each instruction moves two 256-byte rows (lanes 0-15 / 16-31)
           int tr[NI];
@@ -415,7 +524,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           const int stage = (kvc + i) % C::kStages;
           if (!tc_wait(&sm.kv_full[stage], ((kvc + i) / C::kStages) & 1, args.status, abort_flag)) return false;
           const int g = gt + i;
-          const int sb = g & 1, suse = g >> 1;
+          const int sb = g % C::kSBuf, suse = g / C::kSBuf;
           if (suse >= 1 && !tc_wait(&sm.s_free[sb], (suse - 1) & 1, args.status, abort_flag)) return false;
           fence_proxy_async();
           tc_fence_after();
@@ -428,11 +537,15 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           tc_commit(&sm.s_full[sb]);
           return true;
         };
-        if (!issue_qk(0)) { ok = false; break; }
+        // QK runs kSBuf - 1 tiles ahead: QK(i + kSBuf - 1) is issued before PV(i)
+        constexpr int kAhead = C::kSBuf - 1;
+        for (int i0 = 0; i0 < kAhead && i0 < nt; ++i0)
+          if (!issue_qk(i0)) { ok = false; break; }
+        if (!ok) break;
         for (int i = 0; i < nt; ++i) {
-          if (i + 1 < nt && !issue_qk(i + 1)) { ok = false; break; }
+          if (i + kAhead < nt && !issue_qk(i + kAhead)) { ok = false; break; }
           const int g = gt + i;
-          const int pb = g & 1, puse = g >> 1;
+          const int pb = g % C::kSBuf, puse = g / C::kSBuf;
           if (!tc_wait(&sm.p_full[pb], puse & 1, args.status, abort_flag)) { ok = false; break; }
           if (i == 0 && ouse >= 1 && !tc_wait(&sm.o_empty[ob], (ouse - 1) & 1, args.status, abort_flag)) {
             ok = false;
@@ -446,12 +559,12 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           const uint32_t pbase = smem_u32(sm.p[pb]);
 #pragma unroll
           for (int j = 0; j < kTcTile / 16; ++j)
-            mma_bf16(tmem + 2 * N + ob * N, desc_mnmajor(kb, kTcTile * 128, j), desc_mnmajor(pbase, kTcTile * 128, j),
-                     idesc_pv, (i > 0 || j > 0) ? 1u : 0u);
+            mma_bf16(tmem + C::kOCol + ob * N, desc_mnmajor(kb, kTcTile * 128, j),
+                     desc_mnmajor(pbase, kTcTile * 128, j), idesc_pv, (i > 0 || j > 0) ? 1u : 0u);
           if constexpr (C::kSumMma) {
 #pragma unroll
             for (int j = 0; j < kTcTile / 16; ++j)
-              mma_bf16(tmem + 4 * N + ob * N, make_sdesc(ones_base, 128, 256, kLayoutNone),
+              mma_bf16(tmem + C::kLCol + ob * N, make_sdesc(ones_base, 128, 256, kLayoutNone),
                        desc_mnmajor(pbase, kTcTile * 128, j), idesc_sum, (i > 0 || j > 0) ? 1u : 0u);
           }
           tc_commit(&sm.kv_empty[stage]);
@@ -506,9 +619,10 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       }
       named_bar_sync(bar_id, 128);
       bool ok = true;
+      bool tainted = false;   // a clamped softmax argument in this thread (rare)
       for (int i = 0; i < inf.nt; ++i, ++gt) {
-        const int sb = gt & 1;
-        if (!tc_wait(&sm.s_full[sb], (gt >> 1) & 1, args.status, abort_flag)) { ok = false; break; }
+        const int sb = gt % C::kSBuf;
+        if (!tc_wait(&sm.s_full[sb], (gt / C::kSBuf) & 1, args.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (threadIdx.x == 0) CSA_TR(it, i, 4);
         float s[CW];
@@ -570,9 +684,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           }
         }
         // ---- P^T = 2^d (bf16) into shared memory (+ per-thread row sums).
-        // P buffer gt & 1 was last read by PV(gt - 2), which the MMA issued before
-        // QK(gt); s_full(gt) completing implies it completed, so no wait here.
-        const int pb = gt & 1;
+        // P buffer gt % kSBuf was last read by PV(gt - kSBuf), which the MMA
+        // issued before QK(gt); s_full(gt) completing implies it completed.
+        const int pb = gt % C::kSBuf;
         const uint32_t prow = smem_u32(sm.p[pb]) + (col0 >> 6) * (kTcTile * 128) + row * 128;
         auto store_p = [&]() {
 #pragma unroll
@@ -593,7 +707,20 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
                          : "memory");
           }
         };
-        const bool full_max = bar_red_or(bar_id, 128, dmax > 8.0f || newrow);
+        // Once every column has a max (seeded by the sink, or fixed by the
+        // first rows), no group-wide decision is taken per tile: arguments
+        // stay below 2^64 of the max (bf16 / fp32 hold them exactly enough);
+        // a larger one is clamped and the unit is recomputed exactly at its end.
+        bool full_max = false;
+        if (allset) {
+          if (dmax > kClampD) {
+            tainted = true;
+#pragma unroll
+            for (int c = 0; c < CW; ++c) s[c] = fminf(s[c], kClampD);
+          }
+        } else {
+          full_max = bar_red_or(bar_id, 128, dmax > 8.0f || newrow);
+        }
         if (threadIdx.x == 0 && i < 8) CSA_TR(it, 8 + i, 1);
         if (full_max) {
 #pragma unroll
@@ -637,12 +764,15 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           if (rescale) {
             // rare: the running max rose by more than 2^8; PV(i-1) must be complete
             const int gp = gt - 1;
-            if (!tc_wait(&sm.p_empty[gp & 1], (gp >> 1) & 1, args.status, abort_flag)) { ok = false; break; }
+            if (!tc_wait(&sm.p_empty[gp % C::kSBuf], (gp / C::kSBuf) & 1, args.status, abort_flag)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
 #pragma unroll
             for (int buf = 0; buf < (kSumMma ? 2 : 1); ++buf) {
               // O^T, and with the row-sum MMA also L^T, share the column scaling
-              const uint32_t oaddr = tmem + lane_addr + (2 + 2 * buf) * N + ob * N + col0;
+              const uint32_t oaddr = tmem + lane_addr + (buf == 0 ? C::kOCol : C::kLCol) + ob * N + col0;
 #pragma unroll
               for (int h2 = 0; h2 < CW / 16; ++h2) {
                 uint32_t v[16];
@@ -675,8 +805,10 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       // 4-warp total), output scale 2^(m-M) / (l 2^(m-M) + 2^(sigma-M)) with
       // M = max(m, sigma), and lse (natural log, sink excluded)
       if constexpr (!kSumMma) {
+        // butterfly over CW lanes: lane l ends with column l % CW summed over
+        // its CW-lane group; then add the 32 / CW groups
 #pragma unroll
-        for (int st = 16; st >= 1; st >>= 1) {
+        for (int st = CW / 2; st >= 1; st >>= 1) {
           const bool up = (lane & st) != 0;
 #pragma unroll
           for (int e = 0; e < st; ++e) {
@@ -685,7 +817,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
             lpart[e % (kSumMma ? 1 : CW)] = keep + __shfl_xor_sync(0xffffffffu, send, st);
           }
         }
-        sm.xch[wg][wq][lane] = lpart[0];
+#pragma unroll
+        for (int o = CW; o < 32; o <<= 1) lpart[0] += __shfl_xor_sync(0xffffffffu, lpart[0], o);
+        if (lane < CW) sm.xch[wg][wq][lane] = lpart[0];
         named_bar_sync(bar_id, 128);
       }
       if (!tc_wait(&sm.o_full[ob], ouse & 1, args.status, abort_flag)) break;
@@ -697,8 +831,8 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         float l;
         if constexpr (kSumMma) {
           uint32_t v[CW];
-          tmem_ld16(tmem + lane_addr + 4 * N + ob * N + col0, v);   // every lane holds all column sums
-          if constexpr (CW == 32) tmem_ld16(tmem + lane_addr + 4 * N + ob * N + col0 + 16, v + 16);
+          tmem_ld16(tmem + lane_addr + C::kLCol + ob * N + col0, v);   // every lane holds all column sums
+          if constexpr (CW == 32) tmem_ld16(tmem + lane_addr + C::kLCol + ob * N + col0 + 16, v + 16);
           tmem_ld_wait();
           l = 0.f;
 #pragma unroll
@@ -723,11 +857,19 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         const int g = col >> args.hshift;
         if (args.lse != nullptr && lane < CW && g < inf.ntok)
           args.lse[(static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + g) * args.Hq + h] = lse_v;
+        // every weight underflowed although the unit has rows: recompute
+        if (lane < CW && g < inf.ntok && l == 0.f && inf.n_c + inf.n_w > 0) sm.taint[slot] = it + 1;
       }
-      named_bar_sync(bar_id, 128);
+      if (tainted) sm.taint[slot] = it + 1;
+      // all softmax warps: the unit's taint is final after this barrier (the
+      // slot holds the unit's sequence number, so it needs no reset)
+      named_bar_sync(1 + C::kGroups, 128 * C::kGroups);
+      const bool redo = sm.taint[slot] == it + 1;
       if (threadIdx.x == 0) CSA_TR(it, 14, 1);
-      {
-        const uint32_t oaddr = tmem + lane_addr + 2 * N + ob * N + col0;
+      if (redo) {
+        tc_unit_exact(args, inf, sm.sink_l2, N, C::kSoftWarps);
+      } else {
+        const uint32_t oaddr = tmem + lane_addr + C::kOCol + ob * N + col0;
         const int d = row;
         uint32_t v[CW];
         tmem_ld16(oaddr, v);

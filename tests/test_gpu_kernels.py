@@ -438,6 +438,37 @@ def test_attn_rescale_path(ops):
     np.testing.assert_allclose(lse.cpu().numpy(), rl, rtol=0, atol=2.0 ** -8)
 
 
+@pytest.mark.parametrize("case", ["sparse_big_logits", "dense_big_logits", "sparse_sink_dominates"])
+def test_attn_exact_fallback(ops, case):
+    """Units whose softmax arguments leave the fast path's range are recomputed
+    exactly: logits far above the sink (clamped arguments), and a sink so large
+    that every weight underflows (zero row sums)."""
+    B, T, H, D, m, k, W = 1, 400, 64, 128, 4, 48, 128
+    S = T // m
+    q_scale = 60.0 if "big" in case else 1.0
+    q = _randn((B, T, H, D), "bf16", 90, q_scale)
+    kv_c = _randn((B, S, D), "bf16", 91)
+    raw = _randn((B, T, D), "bf16", 92)
+    sink = torch.randn((H,), generator=torch.Generator().manual_seed(93))
+    if case == "sparse_sink_dominates":
+        sink[::2] = 400.0
+    tau = 1 / np.sqrt(D)
+    pos0 = torch.zeros((B,), dtype=torch.int32)
+    pos = np.arange(T)[None]
+    out = torch.empty_like(q, device="cuda")
+    lse = torch.empty((B, T, H), dtype=torch.float32, device="cuda")
+    if case.startswith("sparse"):
+        idx = oracle.topk_select(np.random.default_rng(5).standard_normal((B, T, S)), pos, m, k)
+        ops.sparse_attn_fwd(q.cuda(), kv_c.cuda(), torch.from_numpy(idx).cuda(), raw.cuda(), sink.cuda(), tau, W,
+                            pos0.cuda(), out, lse)
+        ro, rl = oracle.sparse_attn(q, kv_c, idx, raw, T, sink, tau, W, pos)
+    else:
+        ops.hca_dense_attn_fwd(q.cuda(), kv_c.cuda(), raw.cuda(), sink.cuda(), tau, W, pos0.cuda(), out, m, lse=lse)
+        ro, rl = oracle.dense_attn(q, kv_c, raw, T, sink, tau, W, pos, m)
+    _attn_tol("bf16")(_np(out), oracle.round_out(ro, "bf16"))
+    np.testing.assert_allclose(lse.cpu().numpy(), rl, rtol=1e-5, atol=2.0 ** -8)
+
+
 def test_attn_row_chunks_and_empty_sets(ops):
     """row0 > 0 chunks write only their rows; W = 0 rows with no entry give 0."""
     B, T, H, D, m, k, W = 1, 700, 64, 128, 4, 64, 128
