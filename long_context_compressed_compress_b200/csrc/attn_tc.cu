@@ -116,7 +116,6 @@ struct __align__(1024) TcSmem {
   float alpha[C::kGroups][C::kCW];
   float dlt[C::kGroups][C::kCW];
   float sink_l2[128];      // sink logits in log2 units (-inf without a sink)
-  int taint[2];            // unit sequence number + 1 when a unit must be recomputed exactly
   TcUnit info[2];
   uint32_t tmem;
   int abort_flag;
@@ -226,15 +225,15 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, int rows) {
   return (c >> 3) * (rows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
 }
 
-// Exact fallback for one unit, on CUDA cores: every (token, head) column of
-// the unit by one warp at a time (lane = 4 head dims), an online softmax in
+// Exact fallback for columns [col_begin, col_end) of one unit, on CUDA cores:
+// warp w of nw takes every nw-th column (lane = 4 head dims), an online softmax in
 // fp32 over the entries and window rows, then the sink, as the formula states.
 // Used only for units whose fast path was inexact (a logit above the seeded
 // max by more than 2^64, or every weight underflowing).
-__device__ __noinline__ void tc_unit_exact(const TcArgs a, const TcUnit inf, const float* sink_l2, int n_cols,
-                                           int nwarps) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int col = warp; col < n_cols; col += nwarps) {
+__device__ __noinline__ void tc_unit_exact(const TcArgs a, const TcUnit inf, const float* sink_l2, int col_begin,
+                                           int col_end, int w, int nw) {
+  const int lane = threadIdx.x & 31;
+  for (int col = col_begin + w; col < col_end; col += nw) {
     const int g = col >> a.hshift;
     if (g >= inf.ntok) continue;
     const int h = inf.hoff + (col & (a.H - 1));
@@ -324,8 +323,6 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       mbar_init(&sm.p_empty[s], 1);
     }
     sm.abort_flag = 0;
-    sm.taint[0] = 0;
-    sm.taint[1] = 0;
     fence_mbar_init();
   }
   for (int h = threadIdx.x; h < 128; h += blockDim.x)
@@ -825,25 +822,35 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       if (!tc_wait(&sm.o_full[ob], ouse & 1, args.status, abort_flag)) break;
       tc_fence_after();
       if (threadIdx.x == 0) CSA_TR(it, 15, 6);
-      if (wq == 0) {
-        // warp 0 of the warpgroup: lane c < CW handles column col0 + c
-        const int c = lane % CW;
-        float l;
-        if constexpr (kSumMma) {
-          uint32_t v[CW];
-          tmem_ld16(tmem + lane_addr + C::kLCol + ob * N + col0, v);   // every lane holds all column sums
-          if constexpr (CW == 32) tmem_ld16(tmem + lane_addr + C::kLCol + ob * N + col0 + 16, v + 16);
-          tmem_ld_wait();
-          l = 0.f;
+      // Every thread derives its group's CW column scales itself: the column
+      // maxima are in mreg, and the row sums are in every lane of L^T (row-sum
+      // MMA) or in the butterfly totals.  scale = 2^(m-M) / (l 2^(m-M) +
+      // 2^(sigma-M)), M = max(m, sigma); lse = (m + log2 l) ln 2 (sink excluded).
+      float colv[CW];       // row sum, then output scale
+      if constexpr (kSumMma) {
+        uint32_t v[CW];
+        tmem_ld16(tmem + lane_addr + C::kLCol + ob * N + col0, v);
+        if constexpr (CW == 32) tmem_ld16(tmem + lane_addr + C::kLCol + ob * N + col0 + 16, v + 16);
+        tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < CW; ++e)
-            if (e == c) l = __uint_as_float(v[e]);
-        } else {
-          l = (sm.xch[wg][0][c] + sm.xch[wg][1][c]) + (sm.xch[wg][2][c] + sm.xch[wg][3][c]);
-        }
-        const float mcl = mreg[0] * 0.f + sm.mcol[wg][c];
+        for (int c = 0; c < CW; ++c) colv[c] = __uint_as_float(v[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < CW; ++c)
+          colv[c] = (sm.xch[wg][0][c] + sm.xch[wg][1][c]) + (sm.xch[wg][2][c] + sm.xch[wg][3][c]);
+      }
+      bool redo_local = tainted;
+      {
+        // lane c (mod CW) of every warp computes column c once; the CW scales
+        // are then broadcast within the warp with shuffles (no shared memory)
+        const int c = lane % CW;
+        float l = 0.f, mcl = 0.f;
+#pragma unroll
+        for (int e = 0; e < CW; ++e)
+          if (e == c) { l = colv[e]; mcl = mreg[e]; }
         const int col = col0 + c;
         const int h = inf.hoff + (col & (args.H - 1));
+        const bool tok_ok = (col >> args.hshift) < inf.ntok;
         float scale = 0.f, lse_v = -INFINITY;
         if (mcl > 0.5f * kNoRowMax) {
           const float sg = sm.sink_l2[h];
@@ -853,21 +860,19 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           scale = den > 0.f ? __fdiv_rn(f, den) : 0.f;
           if (l > 0.f) lse_v = (mcl + log2f(l)) * 0.6931471805599453f;
         }
-        if (lane < CW) sm.alpha[wg][c] = scale;
-        const int g = col >> args.hshift;
-        if (args.lse != nullptr && lane < CW && g < inf.ntok)
-          args.lse[(static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + g) * args.Hq + h] = lse_v;
         // every weight underflowed although the unit has rows: recompute
-        if (lane < CW && g < inf.ntok && l == 0.f && inf.n_c + inf.n_w > 0) sm.taint[slot] = it + 1;
+        if (tok_ok && l == 0.f && inf.n_c + inf.n_w > 0) redo_local = true;
+        if (wq == 0 && lane < CW && args.lse != nullptr && tok_ok)
+          args.lse[(static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + (col >> args.hshift)) * args.Hq + h] =
+              lse_v;
+#pragma unroll
+        for (int e = 0; e < CW; ++e) colv[e] = __shfl_sync(0xffffffffu, scale, e);
       }
-      if (tainted) sm.taint[slot] = it + 1;
-      // all softmax warps: the unit's taint is final after this barrier (the
-      // slot holds the unit's sequence number, so it needs no reset)
-      named_bar_sync(1 + C::kGroups, 128 * C::kGroups);
-      const bool redo = sm.taint[slot] == it + 1;
+      // group-wide decision; a tainted group recomputes its own columns exactly
+      const bool redo = bar_red_or(bar_id, 128, redo_local);
       if (threadIdx.x == 0) CSA_TR(it, 14, 1);
       if (redo) {
-        tc_unit_exact(args, inf, sm.sink_l2, N, C::kSoftWarps);
+        tc_unit_exact(args, inf, sm.sink_l2, col0, col0 + CW, wq, 4);
       } else {
         const uint32_t oaddr = tmem + lane_addr + C::kOCol + ob * N + col0;
         const int d = row;
@@ -882,7 +887,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         for (int c = 0; c < CW; ++c) {
           const int col = col0 + c;
           if ((col >> args.hshift) >= inf.ntok) continue;
-          obase[static_cast<size_t>(col) * kTcDim] = __float2bfloat16_rn(__uint_as_float(v[c]) * sm.alpha[wg][c]);
+          obase[static_cast<size_t>(col) * kTcDim] = __float2bfloat16_rn(__uint_as_float(v[c]) * colv[c]);
         }
       }
       if (threadIdx.x == 0) CSA_TR(it, 14, 3);
