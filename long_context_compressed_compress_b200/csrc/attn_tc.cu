@@ -170,6 +170,16 @@ __device__ __forceinline__ float fast_ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
+__device__ __forceinline__ float fast_rcp(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float fast_lg2(float x) {
+  float r;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 // d = a * b + c and x += y on pairs of floats (packed f32x2 pipe ops).
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
                                       float c1) {
@@ -853,12 +863,14 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         const bool tok_ok = (col >> args.hshift) < inf.ntok;
         float scale = 0.f, lse_v = -INFINITY;
         if (mcl > 0.5f * kNoRowMax) {
+          // approximate ex2 / rcp / lg2 (relative error ~2^-22) are ample for a
+          // bf16 output and an fp32 lse
           const float sg = sm.sink_l2[h];
           const float mx = fmaxf(mcl, sg);
-          const float f = exp2f(mcl - mx);
-          const float den = fmaf(l, f, exp2f(sg - mx));
-          scale = den > 0.f ? __fdiv_rn(f, den) : 0.f;
-          if (l > 0.f) lse_v = (mcl + log2f(l)) * 0.6931471805599453f;
+          const float f = fast_ex2(mcl - mx);
+          const float den = fmaf(l, f, fast_ex2(sg - mx));
+          scale = den > 0.f ? f * fast_rcp(den) : 0.f;
+          if (l > 0.f) lse_v = (mcl + fast_lg2(l)) * 0.6931471805599453f;
         }
         // every weight underflowed although the unit has rows: recompute
         if (tok_ok && l == 0.f && inf.n_c + inf.n_w > 0) redo_local = true;
@@ -883,11 +895,23 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         if (threadIdx.x == 0) CSA_TR(it, 14, 2);
         __nv_bfloat16* obase =
             args.out + ((static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0) * args.Hq + inf.hoff) * kTcDim + d;
+        // lane pairs trade half their columns so that each lane holds two
+        // adjacent head dims of CW/2 columns: the even lane columns [0, CW/2)
+        // at dims (d, d + 1), the odd lane columns [CW/2, CW) at (d - 1, d);
+        // then one 4-byte bf16x2 store per column
+        constexpr int HC = CW / 2;
+        const bool odd = (lane & 1) != 0;
+        __nv_bfloat16* pbase = obase - (odd ? 1 : 0);
 #pragma unroll
-        for (int c = 0; c < CW; ++c) {
+        for (int j = 0; j < HC; ++j) {
+          const float lo = __uint_as_float(v[j]) * colv[j];
+          const float hi = __uint_as_float(v[HC + j]) * colv[HC + j];
+          const float recv = __shfl_xor_sync(0xffffffffu, odd ? lo : hi, 1);
+          const int c = odd ? HC + j : j;
           const int col = col0 + c;
-          if ((col >> args.hshift) >= inf.ntok) continue;
-          obase[static_cast<size_t>(col) * kTcDim] = __float2bfloat16_rn(__uint_as_float(v[c]) * colv[c]);
+          const uint32_t w = odd ? pack_bf16(recv, hi) : pack_bf16(lo, recv);
+          if ((col >> args.hshift) < inf.ntok)
+            *reinterpret_cast<uint32_t*>(pbase + static_cast<size_t>(col) * kTcDim) = w;
         }
       }
       if (threadIdx.x == 0) CSA_TR(it, 14, 3);
