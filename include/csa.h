@@ -208,8 +208,8 @@ int topk_select_noalloc(const void* score, int score_dtype, int B, int T_chunk,
  *   kv_c [B, kv_bstride, D], idx int32 [B, T_chunk, k] (each row: its valid
  *   entries first, then -1 padding, as topk_select writes it), kv_raw [B, raw_cap, D]
  *   sink fp32 [H] or NULL, lse fp32 [B, T, H] or NULL
- * Requires D in {64, 128}; bf16 runs on tcgen05 (H in {16..128}, H % 16 == 0),
- * fp32 on CUDA cores in fp32.
+ * Requires D in {64, 128}.  bf16 runs on tcgen05 and needs D = 128, H in
+ * {64, 128} and k <= 1024 (else CSA_ERR_UNSUPPORTED); fp32 runs on CUDA cores.
  */
 int sparse_attn_fwd(const void* q, const void* kv_c, const int32_t* idx,
                     const void* kv_raw, const float* sink, float tau, int W,
@@ -222,6 +222,7 @@ int sparse_attn_fwd(const void* q, const void* kv_c, const int32_t* idx,
  * compressed entries, no selection; §3.3 window and sink): as sparse_attn_fwd
  * with the entry set = every visible entry s < S (m*(s+1) - 1 <= p).
  *   kv_c [B, kv_bstride, D]
+ * bf16 needs D = 128 and H in {16, 32, 64, 128}; fp32 runs on CUDA cores.
  */
 int hca_dense_attn_fwd(const void* q, const void* kv_c, const void* kv_raw,
                        const float* sink, float tau, int W,

@@ -975,8 +975,9 @@ int launch_attn_tc_nb(const TcArgs& a, const TcMaps& maps, cudaStream_t st) {
   return check_launch();
 }
 
-// bf16 tcgen05 attention.  Requirements: D == 128, and N = G*H in {64, 128}
-// with G = 1 for sparse (CSA) units; for dense (HCA) units G = 128 / H.
+// bf16 tcgen05 attention.  Requirements: D == 128; every call runs units of
+// N = G*H = 64 columns: G = 1 token of 64 heads (128 heads split in two), or
+// for dense (HCA) calls with H < 64, G = 64 / H tokens sharing the entries.
 int launch_attn_tc(const void* q, const void* kv_c, const int32_t* idx, const void* kv_raw, const float* sink,
                    float tau, int W, int B, int Tq, int row0, int T_chunk, int H, int kv_bstride, int k, int S, int m,
                    int raw_cap, const int32_t* q_pos0, void* out, float* lse, int sparse, cudaStream_t st) {
@@ -985,16 +986,17 @@ int launch_attn_tc(const void* q, const void* kv_c, const int32_t* idx, const vo
     CSA_REQUIRE(H == 64 || H == 128, CSA_ERR_UNSUPPORTED);
   } else {
     CSA_REQUIRE(H == 16 || H == 32 || H == 64 || H == 128, CSA_ERR_UNSUPPORTED);
-    G = 128 / H;
+    G = H < 64 ? 64 / H : 1;     // units of N = 64 (token, head) columns
   }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // Few query rows (decode): split 128 heads into two 64-head units, which
-  // doubles the CTAs at work and uses the N = 64 tile; the extra gather of the
-  // same KV rows is small when there are few rows.
+  // 128 heads run as two 64-head units of one token each: the N = 64 tile
+  // (three S / P buffers, 80 registers without spilling its softmax loop) beats
+  // the N = 128 tile even though each KV tile is fetched twice (from L2)
   const int Hq = H;
-  const int hsplit = (sparse && H == 128 && static_cast<long long>(B) * T_chunk < sms) ? 2 : 1;
+  const int hsplit = H == 128 ? 2 : 1;
+  if (hsplit == 2) G = 1;
   H = Hq / hsplit;
   const int N = G * H;
   TcArgs a;
@@ -1034,7 +1036,8 @@ int launch_attn_tc(const void* q, const void* kv_c, const int32_t* idx, const vo
       !make_map(&maps.raw, kv_raw ? kv_raw : kv_c, static_cast<uint64_t>(kv_raw ? raw_rows : kv_rows), kTcTile))
     return CSA_ERR_CUDA;
   if (!kv_raw) a.raw_rows = a.kv_rows;
-  return N == 64 ? launch_attn_tc_nb<1>(a, maps, st) : launch_attn_tc_nb<2>(a, maps, st);
+  CSA_REQUIRE(N == 64, CSA_ERR_UNSUPPORTED);
+  return launch_attn_tc_nb<1>(a, maps, st);
 }
 
 }  // namespace csa
