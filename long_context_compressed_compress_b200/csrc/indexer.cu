@@ -5,8 +5,9 @@
 //   score[t, s] = sum_h w[t,h] * ReLU( qhat[t,h,:] . khat[s,:] )
 //
 // The contraction runs "entries x (token, head)": the MMA's M = 128 compressed
-// entries, N = 128 (token, head) pairs (128/HI tokens x HI heads), K = 64 FP4
-// values (one MMA; DI = 32 is zero-padded).  The accumulator tile lives in
+// entries, N (token, head) pairs (N/HI tokens x HI heads; N = 112 for prefill
+// chunks, 16 for decode chunks), K = 64 FP4 values (one MMA; DI = 32 is
+// zero-padded).  The accumulator tile lives in
 // TMEM with one entry per lane, so each epilogue thread owns one entry and the
 // HI heads of a token sit in adjacent columns of its own lane: the weighted
 // ReLU head-sum needs no cross-thread reduction, and the 32 threads of a warp
@@ -15,8 +16,8 @@
 // folded into w.  Operands are staged with cp.async into the canonical
 // no-swizzle K-major layout (8 rows x 16 B core matrices).
 //
-// A CTA owns one tile of 128 (token, head) rows and up to kTilesPerCta entry
-// tiles; entry tiles are double-buffered in shared memory.  Work above the
+// A CTA owns one tile of N (token, head) rows and up to kTilesPerCta entry
+// tiles, streamed through a ring of shared-memory stages.  Work above the
 // causal limit (entries no query of the tile can see) is never launched.
 #include "common.cuh"
 
@@ -26,12 +27,16 @@ constexpr int kIdxThreads = 128;
 // entry tiles per CTA and shared-memory stages: the narrow (decode) tile
 // streams more tiles per CTA through a deeper ring
 template <int NQ> struct IdxShape {
-  static constexpr int tiles = NQ == 128 ? 8 : 16;
-  static constexpr int stages = NQ == 128 ? 2 : 4;
+  static constexpr int tiles = NQ > 16 ? 8 : 16;
+  static constexpr int stages = NQ > 16 ? 2 : 4;
 };
 // TMEM columns: accumulator NQ + SFA 4 + SFB 4, rounded to a power of two
-template <int NQ> struct IdxTmem { static constexpr uint32_t cols = NQ == 128 ? 256 : 32; };
-constexpr size_t kIdxSmemFloor = 96 * 1024;  // keeps <= 2 CTAs per SM (TMEM 2 x 256 cols)
+template <int NQ> struct IdxTmem { static constexpr uint32_t cols = NQ + 8 <= 32 ? 32 : (NQ + 8 <= 128 ? 128 : 256); };
+// shared-memory floor per CTA so that no more CTAs share an SM than its 512
+// TMEM columns hold (a CTA waiting in tcgen05.alloc would only idle)
+template <int NQ> struct IdxFloor {
+  static constexpr size_t bytes = IdxTmem<NQ>::cols == 256 ? 96 * 1024 : (IdxTmem<NQ>::cols == 128 ? 48 * 1024 : 0);
+};
 
 template <int NS>
 struct __align__(128) IdxSmem {
@@ -173,7 +178,7 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
     // ---- epilogue: this thread owns entry s; columns are (token, head) pairs
     const int s = (et0 + j) * 128 + tid;
     const bool s_ok = s < S;
-    constexpr int CB = NQ < 32 ? NQ : 32;      // columns per TMEM load
+    constexpr int CB = NQ % 32 == 0 ? 32 : 16;   // columns per TMEM load
 #pragma unroll 1
     for (int c0 = 0; c0 < NQ; c0 += CB) {
       uint32_t v[CB];
@@ -217,16 +222,20 @@ extern "C" int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_
   CSA_REQUIRE(aligned16(q_fp4) && aligned16(k_fp4), CSA_ERR_ALIGNMENT);
   CSA_REQUIRE(DI != 64 || (reinterpret_cast<uintptr_t>(k_sf) & 3) == 0, CSA_ERR_ALIGNMENT);
   if (B == 0 || T_chunk == 0 || S == 0) return CSA_OK;
-  const bool narrow = T_chunk * HI <= 16;      // decode-sized chunk: N = 16
-  const int TQ = (narrow ? 16 : 128) / HI;
+  // N = 16 for decode-sized chunks; N = 112 (TMEM 128 columns, four CTAs per
+  // SM) for prefill chunks
+  const bool narrow = T_chunk * HI <= 16;
+  constexpr int kWide = 112;
+  const int TQ = (narrow ? 16 : kWide) / HI;
   const int n_qtiles = (T_chunk + TQ - 1) / TQ;
   const int n_et = (S + 127) / 128;
-  const int tiles_per_cta = narrow ? IdxShape<16>::tiles : IdxShape<128>::tiles;
+  const int tiles_per_cta = narrow ? IdxShape<16>::tiles : IdxShape<kWide>::tiles;
   const int n_chunks = (n_et + tiles_per_cta - 1) / tiles_per_cta;
   const long long grid = static_cast<long long>(B) * n_qtiles * n_chunks;
   CSA_REQUIRE(grid < (1ll << 31), CSA_ERR_UNSUPPORTED);
-  const size_t smem_min = (narrow ? sizeof(IdxSmem<IdxShape<16>::stages>) : sizeof(IdxSmem<IdxShape<128>::stages>)) + 1024;
-  const size_t smem = narrow ? smem_min : (smem_min > kIdxSmemFloor ? smem_min : kIdxSmemFloor);
+  const size_t smem_min = (narrow ? sizeof(IdxSmem<IdxShape<16>::stages>) : sizeof(IdxSmem<IdxShape<kWide>::stages>)) + 1024;
+  const size_t floor_b = narrow ? IdxFloor<16>::bytes : IdxFloor<kWide>::bytes;
+  const size_t smem = smem_min > floor_b ? smem_min : floor_b;
   const float g = q_gscale * k_gscale;
   int* status = device_status_ptr();
   CSA_REQUIRE(status != nullptr, CSA_ERR_CUDA);
@@ -242,7 +251,7 @@ extern "C" int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_
 #define CSA_IDX_LAUNCH(HIV, TS)                                 \
   do {                                                          \
     if (narrow) CSA_IDX_LAUNCH_NQ(HIV, TS, 16);                 \
-    else CSA_IDX_LAUNCH_NQ(HIV, TS, 128);                       \
+    else CSA_IDX_LAUNCH_NQ(HIV, TS, kWide);                     \
   } while (0)
 #define CSA_IDX_DT(HIV)                                                \
   do {                                                                 \
