@@ -237,10 +237,61 @@ __host__ __device__ __forceinline__ void run_shape(int n, int* L, int* Lp) {
   *Lp = ((l / V) & 1) ? l : l + V;
 }
 
+// Radix select over 16-bit keys held in registers (kk[0, cntp) per thread):
+// the key value K of the r-th largest (1 <= r <= total) and krem = r - #(> K).
+template <int NT, int MAXP>
+__device__ __forceinline__ void block_select16(const uint32_t (&kk)[MAXP], int cntp, int r, int* hflat, int* wsum,
+                                               int* sel_digit, int* sel_above, uint32_t* K_out, int* krem_out) {
+  constexpr int DPT = (256 + NT - 1) / NT;
+  const int tid = threadIdx.x;
+  const int cp = tid & (kRunCopies - 1);
+  uint32_t prefix = 0, pmask = 0;
+  int krem = r;
+#pragma unroll 1
+  for (int shift = 8; shift >= 0; shift -= 8) {
+    for (int i = tid; i < kRunCopies * 256; i += NT) hflat[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < MAXP; ++q)
+      if (q < cntp && (kk[q] & pmask) == prefix) atomicAdd(&hflat[cp * 256 + ((kk[q] >> shift) & 0xFFu)], 1);
+    __syncthreads();
+    int cq[DPT], csum = 0;
+#pragma unroll
+    for (int q = 0; q < DPT; ++q) {
+      const int d = 255 - DPT * tid - q;
+      int c = 0;
+      if (d >= 0) {
+#pragma unroll
+        for (int c2 = 0; c2 < kRunCopies; ++c2) c += hflat[c2 * 256 + d];
+      }
+      cq[q] = c;
+      csum += c;
+    }
+    int tot;
+    int above = block_excl_scan_nt<NT>(csum, wsum, &tot);
+#pragma unroll
+    for (int q = 0; q < DPT; ++q) {
+      if (above < krem && krem <= above + cq[q]) {
+        *sel_digit = 255 - DPT * tid - q;
+        *sel_above = above;
+      }
+      above += cq[q];
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(*sel_digit) << shift;
+    pmask |= 0xFFu << shift;
+    krem -= *sel_above;
+  }
+  *K_out = prefix;
+  *krem_out = krem;
+}
+
+constexpr int kCandCap = 2048;   // candidates a sampled threshold may admit
+
 template <typename T, int NT>
 __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ score, int T_chunk, int S, int ld,
                                                       int k, int m, int row0, const int32_t* __restrict__ q_pos0,
-                                                      int32_t* __restrict__ idx) {
+                                                      int32_t* __restrict__ idx, int cand_off) {
   using KO = KeyOf<T>;
   using K = typename KO::K;
   static_assert(sizeof(K) == sizeof(T), "key and score widths match");
@@ -273,6 +324,12 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
   for (int i = tid; i < kRunCopies * 256; i += NT) hflat[i] = 0;
   __syncthreads();
 
+  // rows that try the sampled threshold first take their first-digit
+  // histogram only if they fall back to the full radix path
+  // (long rows only: on short rows the two small selects cost more than the
+  // radix passes they save)
+  const bool sampled = KO::bits == 16 && NT >= 512 && n >= 2 * k && n > 4 * NT;
+  const bool hist_in_load = !sampled;
   // ---- stage the row as keys (16-byte loads where aligned) + first-digit histogram
   const T* srow = score + static_cast<size_t>(row) * ld;
   int done = 0;
@@ -286,7 +343,7 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
 #pragma unroll
       for (int q = 0; q < V; ++q) {
         kk[q] = KO::get(e[q]);
-        atomicAdd(&hist[cp][static_cast<uint32_t>(kk[q]) >> top], 1);
+        if (hist_in_load) atomicAdd(&hist[cp][static_cast<uint32_t>(kk[q]) >> top], 1);
       }
       const int i = g * V;
       const int t = i / L;
@@ -297,7 +354,7 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
   }
   for (int i = done + tid; i < n; i += NT) {
     const K key = KO::get(srow[i]);
-    atomicAdd(&hist[cp][static_cast<uint32_t>(key) >> top], 1);
+    if (hist_in_load) atomicAdd(&hist[cp][static_cast<uint32_t>(key) >> top], 1);
     const int t = i / L;
     keys[static_cast<size_t>(t) * Lp + (i - t * L)] = key;
   }
@@ -305,6 +362,104 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
 
   const int cnt = max(0, min(L, n - tid * L));
   const K* run = keys + static_cast<size_t>(tid) * Lp;
+
+  if constexpr (KO::bits == 16 && NT >= 512) {
+    // ---- sampled threshold (long rows with n >= 2k): a radix select over 4 NT
+    // evenly spaced keys gives T0, about 1.25 k + n / NT keys of the row lie
+    // at or above it.  If at least k and at most kCandCap do, those candidates
+    // are compacted in index order and the exact selection runs on them alone
+    // (every key of the top k is >= T0 when at least k keys are); otherwise
+    // the row takes the full radix path below.
+    if (sampled) {
+      constexpr int SPT = 4;                  // samples per thread
+      constexpr int kSamples = SPT * NT;
+      uint32_t sk[SPT];
+#pragma unroll
+      for (int q = 0; q < SPT; ++q) {
+        const int pos = static_cast<int>(static_cast<long long>(tid * SPT + q) * n / kSamples);
+        const int t = pos / L;
+        sk[q] = keys[static_cast<size_t>(t) * Lp + (pos - t * L)];
+      }
+      int r = static_cast<int>(static_cast<long long>(5 * k) * kSamples / (4ll * n)) + 4;
+      if (r > kSamples) r = kSamples;
+      uint32_t T0;
+      int unused;
+      block_select16<NT, SPT>(sk, SPT, r, hflat, wsum, &sel_digit, &sel_above, &T0, &unused);
+      int nge = 0;
+      for (int j = 0; j < cnt; j += V) {
+        const uint4 u = *reinterpret_cast<const uint4*>(run + j);
+        const K* kk = reinterpret_cast<const K*>(&u);
+#pragma unroll
+        for (int q = 0; q < V; ++q) nge += (j + q < cnt && static_cast<uint32_t>(kk[q]) >= T0);
+      }
+      int tot;
+      int cpos = block_excl_scan_nt<NT>(nge, wsum, &tot);
+      if (tot >= k && tot <= kCandCap) {
+        uint16_t* ckey = reinterpret_cast<uint16_t*>(dsm + cand_off);
+        int32_t* cidx = reinterpret_cast<int32_t*>(dsm + cand_off + kCandCap * 2);
+        const int base = tid * L;
+        for (int j = 0; j < cnt; j += V) {
+          const uint4 u = *reinterpret_cast<const uint4*>(run + j);
+          const K* kk = reinterpret_cast<const K*>(&u);
+#pragma unroll
+          for (int q = 0; q < V; ++q) {
+            const uint32_t key = kk[q];
+            if (j + q < cnt && key >= T0) {
+              ckey[cpos] = static_cast<uint16_t>(key);
+              cidx[cpos] = base + j + q;
+              ++cpos;
+            }
+          }
+        }
+        __syncthreads();
+        // exact selection among the tot candidates (index order): thread t owns
+        // candidates [t cpt, t cpt + cpt)
+        constexpr int CPT = kCandCap / NT;
+        const int cpt = (tot + NT - 1) / NT;
+        const int c0 = tid * cpt;
+        const int cc = max(0, min(cpt, tot - c0));
+        uint32_t ck[CPT];
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) ck[q] = q < cc ? ckey[c0 + q] : 0u;
+        uint32_t Kf;
+        int kremf;
+        block_select16<NT, CPT>(ck, cc, k, hflat, wsum, &sel_digit, &sel_above, &Kf, &kremf);
+        int n_gt = 0, n_eq = 0;
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) {
+          n_gt += q < cc && ck[q] > Kf;
+          n_eq += q < cc && ck[q] == Kf;
+        }
+        int tg, te;
+        const int gt_before = block_excl_scan_nt<NT>(n_gt, wsum, &tg);
+        int eq_seen = block_excl_scan_nt<NT>(n_eq, wsum, &te);
+        int pos = gt_before + min(eq_seen, kremf);
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) {
+          if (q < cc) {
+            if (ck[q] > Kf) {
+              out[pos++] = cidx[c0 + q];
+            } else if (ck[q] == Kf) {
+              if (eq_seen < kremf) out[pos++] = cidx[c0 + q];
+              ++eq_seen;
+            }
+          }
+        }
+        return;
+      }
+      // fall back to the full radix path: take its first-digit histogram now
+      for (int i = tid; i < kRunCopies * 256; i += NT) hflat[i] = 0;
+      __syncthreads();
+      for (int j = 0; j < cnt; j += V) {
+        const uint4 u = *reinterpret_cast<const uint4*>(run + j);
+        const K* kk = reinterpret_cast<const K*>(&u);
+#pragma unroll
+        for (int q = 0; q < V; ++q)
+          if (j + q < cnt) atomicAdd(&hist[cp][static_cast<uint32_t>(kk[q]) >> top], 1);
+      }
+      __syncthreads();
+    }
+  }
   uint32_t prefix = 0, pmask = 0;
   int krem = k;
 #pragma unroll 1
@@ -387,13 +542,18 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
   }
 }
 
+// keys region, then (16-bit keys) the candidate buffer of the sampled path
 template <typename T, int NT>
-size_t run_smem_bytes(int S) {
+size_t run_keys_bytes(int S) {
   using K = typename KeyOf<T>::K;
   constexpr int V = 16 / sizeof(K);
   int L, Lp;
   run_shape<NT, V>(S, &L, &Lp);
-  return static_cast<size_t>(NT) * (L + V) * sizeof(K);
+  return (static_cast<size_t>(NT) * (L + V) * sizeof(K) + 15) & ~static_cast<size_t>(15);
+}
+template <typename T, int NT>
+size_t run_smem_bytes(int S) {
+  return run_keys_bytes<T, NT>(S) + (KeyOf<T>::bits == 16 && NT >= 512 ? static_cast<size_t>(kCandCap) * 6 : 0);
 }
 
 template <typename T, int NT>
@@ -407,8 +567,8 @@ int launch_topk_run(const T* score, long long rows, int T_chunk, int S, int ld, 
     if (e != cudaSuccess) return set_cuda_error(e);
     attr = static_cast<int>(kTopkSmemMax);
   }
-  topk_run_kernel<T, NT><<<static_cast<unsigned>(rows), NT, bytes, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0,
-                                                                         idx);
+  topk_run_kernel<T, NT><<<static_cast<unsigned>(rows), NT, bytes, st>>>(
+      score, T_chunk, S, ld, k, m, row0, q_pos0, idx, static_cast<int>(run_keys_bytes<T, NT>(S)));
   return check_launch();
 }
 
