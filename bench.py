@@ -44,7 +44,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--chunk", type=int, default=0, help="query rows per indexer/top-k chunk (0 = all)")
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--cpu-rows", type=int, default=96, help="query rows in the CPU-oracle sample")
+    ap.add_argument("--cpu-rows", type=int, default=4096, help="query rows in the CPU-oracle sample (about 10 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=0,
                     help="profiling case: override the layer's token count (not a bench line)")
