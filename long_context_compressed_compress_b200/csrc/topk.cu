@@ -641,6 +641,25 @@ __device__ __forceinline__ void mc_find_bin(const int* h, int krem, int* wsum, i
   __syncthreads();
 }
 
+// Keys [i, i + 8) of a row as order-preserving keys (valid where < i1): one
+// 16-byte load when the row start is 16-byte aligned and the load stays inside
+// the row's ld elements, else element loads.
+__device__ __forceinline__ void mc_load8(const __nv_bfloat16* srow, int i, int i1, int ld, bool aligned,
+                                         uint32_t (&kk)[8]) {
+  using KO = KeyOf<__nv_bfloat16>;
+  if (aligned && i + 8 <= ld) {
+    const uint4 u = *reinterpret_cast<const uint4*>(srow + i);
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) kk[q] = KO::get(e[q]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) kk[q] = i + q < i1 ? static_cast<uint32_t>(KO::get(srow[i + q])) : 0u;
+  }
+}
+// thread t of a chunk owns keys [i0 + kMcRun t, i0 + kMcRun (t + 1))
+constexpr int kMcRun = kMcChunk / kMcThreads;   // 32
+
 __global__ void __launch_bounds__(kMcThreads) topk_mc_hist1(const __nv_bfloat16* __restrict__ score, int T_chunk,
                                                             int S, int ld, int k, int m, int row0,
                                                             const int32_t* __restrict__ q_pos0, int* __restrict__ ws) {
@@ -655,7 +674,19 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_hist1(const __nv_bfloat16*
   for (int i = threadIdx.x; i < kMcHist1; i += kMcThreads) h[i] = 0;
   __syncthreads();
   const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
-  for (int i = i0 + threadIdx.x; i < i1; i += kMcThreads) atomicAdd(&h[KO::get(srow[i]) >> 5], 1);
+  const bool al = (reinterpret_cast<uintptr_t>(srow) & 15) == 0;
+  const int r0 = i0 + kMcRun * threadIdx.x;
+#pragma unroll
+  for (int g = 0; g < kMcRun / 8; ++g) {
+    const int b = r0 + 8 * g;
+    if (b < i1) {
+      uint32_t kk[8];
+      mc_load8(srow, b, i1, ld, al, kk);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (b + q < i1) atomicAdd(&h[kk[q] >> 5], 1);
+    }
+  }
   __syncthreads();
   int* g = ws + static_cast<size_t>(row) * L.row_ints;
   for (int i = threadIdx.x; i < kMcHist1; i += kMcThreads)
@@ -686,9 +717,18 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_hist2(const __nv_bfloat16*
   }
   const int i0 = c * kMcChunk, i1 = min(n, i0 + kMcChunk);
   const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
-  for (int i = i0 + threadIdx.x; i < i1; i += kMcThreads) {
-    const uint32_t key = KO::get(srow[i]);
-    if (static_cast<int>(key >> 5) == b1) atomicAdd(&h2[key & 31], 1);
+  const bool al = (reinterpret_cast<uintptr_t>(srow) & 15) == 0;
+  const int r0 = i0 + kMcRun * threadIdx.x;
+#pragma unroll
+  for (int g = 0; g < kMcRun / 8; ++g) {
+    const int b = r0 + 8 * g;
+    if (b < i1) {
+      uint32_t kk[8];
+      mc_load8(srow, b, i1, ld, al, kk);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (b + q < i1 && static_cast<int>(kk[q] >> 5) == b1) atomicAdd(&h2[kk[q] & 31], 1);
+    }
   }
   __syncthreads();
   if (threadIdx.x < kMcHist2 && h2[threadIdx.x]) atomicAdd(&g[McLayout::kHist2 + threadIdx.x], h2[threadIdx.x]);
@@ -720,11 +760,21 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_count(const __nv_bfloat16*
   }
   const int i0 = c * kMcChunk, i1 = min(n, i0 + kMcChunk);
   const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
+  const bool al = (reinterpret_cast<uintptr_t>(srow) & 15) == 0;
+  const int r0 = i0 + kMcRun * threadIdx.x;
   int n_gt = 0, n_eq = 0;
-  for (int i = i0 + threadIdx.x; i < i1; i += kMcThreads) {
-    const uint32_t key = KO::get(srow[i]);
-    n_gt += key > K;
-    n_eq += key == K;
+#pragma unroll
+  for (int g = 0; g < kMcRun / 8; ++g) {
+    const int b = r0 + 8 * g;
+    if (b < i1) {
+      uint32_t kk[8];
+      mc_load8(srow, b, i1, ld, al, kk);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        n_gt += b + q < i1 && kk[q] > K;
+        n_eq += b + q < i1 && kk[q] == K;
+      }
+    }
   }
   n_gt = __reduce_add_sync(0xffffffffu, n_gt);
   n_eq = __reduce_add_sync(0xffffffffu, n_eq);
@@ -743,8 +793,7 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_emit(const __nv_bfloat16* 
                                                            int S, int ld, int k, int m, int row0,
                                                            const int32_t* __restrict__ q_pos0,
                                                            const int* __restrict__ ws, int32_t* __restrict__ idx) {
-  using KO = KeyOf<__nv_bfloat16>;
-  __shared__ int wcnt[kMcWarps][2];
+  __shared__ int wsum[kMcWarps];
   const McLayout L(S);
   const int row = blockIdx.x / L.C, c = blockIdx.x % L.C;
   const int n = mc_row_n(row, T_chunk, S, m, row0, q_pos0);
@@ -761,41 +810,52 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_emit(const __nv_bfloat16* 
   const int* g = ws + static_cast<size_t>(row) * L.row_ints;
   const uint32_t K = static_cast<uint32_t>(g[McLayout::kState + 2]);
   const int krem = g[McLayout::kState + 3];
-  int out_pos = 0, eq_before = 0;
+  // keys > K and == K in the chunks before this one
+  int gt_c = 0, eq_c = 0;
   for (int cc = 0; cc < c; ++cc) {
-    const int gt = g[McLayout::kCnt + 2 * cc], eq = g[McLayout::kCnt + 2 * cc + 1];
-    out_pos += gt + max(0, min(eq, krem - eq_before));
-    eq_before += eq;
+    gt_c += g[McLayout::kCnt + 2 * cc];
+    eq_c += g[McLayout::kCnt + 2 * cc + 1];
   }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // this thread's run, then its output position: every key > K before it in
+  // the row, plus the keys == K before it that are taken (the first krem)
   const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
-  const int seg = kMcChunk / kMcWarps;
-  const int s0 = i0 + warp * seg, s1 = min(i1, s0 + seg);
+  const bool al = (reinterpret_cast<uintptr_t>(srow) & 15) == 0;
+  const int r0 = i0 + kMcRun * threadIdx.x;
+  uint32_t kr[kMcRun];
+#pragma unroll
+  for (int gq = 0; gq < kMcRun / 8; ++gq) {
+    uint32_t kk[8];
+    const int b = r0 + 8 * gq;
+    if (b < i1) {
+      mc_load8(srow, b, i1, ld, al, kk);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) kk[q] = 0u;
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) kr[8 * gq + q] = kk[q];
+  }
   int n_gt = 0, n_eq = 0;
-  for (int b0 = s0; b0 < s1; b0 += 32) {
-    const int i = b0 + lane;
-    const uint32_t key = i < s1 ? static_cast<uint32_t>(KO::get(srow[i])) : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, i < s1 && key > K));
-    n_eq += __popc(__ballot_sync(0xffffffffu, i < s1 && key == K));
+#pragma unroll
+  for (int q = 0; q < kMcRun; ++q) {
+    n_gt += r0 + q < i1 && kr[q] > K;
+    n_eq += r0 + q < i1 && kr[q] == K;
   }
-  if (lane == 0) { wcnt[warp][0] = n_gt; wcnt[warp][1] = n_eq; }
-  __syncthreads();
-  for (int w = 0; w < warp; ++w) {
-    out_pos += wcnt[w][0] + max(0, min(wcnt[w][1], krem - eq_before));
-    eq_before += wcnt[w][1];
-  }
-  const unsigned below = (1u << lane) - 1u;
-  for (int b0 = s0; b0 < s1; b0 += 32) {
-    const int i = b0 + lane;
-    const uint32_t key = i < s1 ? static_cast<uint32_t>(KO::get(srow[i])) : 0u;
-    const bool gt = i < s1 && key > K;
-    const bool eq = i < s1 && key == K;
-    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-    const bool take = gt || (eq && eq_before + __popc(eqm & below) < krem);
-    const unsigned tm = __ballot_sync(0xffffffffu, take);
-    if (take) out[out_pos + __popc(tm & below)] = i;
-    out_pos += __popc(tm);
-    eq_before += __popc(eqm);
+  int tg, te;
+  const int gt_t = block_excl_scan_nt<kMcThreads>(n_gt, wsum, &tg);
+  int eq_seen = eq_c + block_excl_scan_nt<kMcThreads>(n_eq, wsum, &te);
+  int pos = gt_c + gt_t + min(eq_seen, krem);
+#pragma unroll
+  for (int q = 0; q < kMcRun; ++q) {
+    const int i = r0 + q;
+    if (i < i1) {
+      if (kr[q] > K) {
+        out[pos++] = i;
+      } else if (kr[q] == K) {
+        if (eq_seen < krem) out[pos++] = i;
+        ++eq_seen;
+      }
+    }
   }
 }
 

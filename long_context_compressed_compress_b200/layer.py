@@ -164,7 +164,8 @@ class CsaDecode:
         self.q_fp4 = torch.empty((B, 1, c.HI, c.DI // 2), dtype=torch.uint8, device=device)
         self.q_sf = torch.empty((B, 1, c.HI, c.DI // 16), dtype=torch.uint8, device=device)
         sdt = torch.float32 if c.dtype == "f32" else torch.bfloat16
-        self.score = torch.empty((B, 1, cap), dtype=sdt, device=device)
+        # row stride padded to 8 elements so every score row is 16-byte aligned
+        self.score = torch.empty((B, 1, (cap + 7) // 8 * 8), dtype=sdt, device=device)
         self.idx = torch.empty((B, 1, c.k), dtype=torch.int32, device=device)
         self.out = torch.empty((B, 1, c.H, D), dtype=dt, device=device)
         self.lse = torch.empty((B, 1, c.H), dtype=torch.float32, device=device) if with_lse else None
