@@ -66,25 +66,21 @@ struct TcCfg {
   static constexpr int kCW = NB == 1 ? 16 : 32;            // columns per softmax warpgroup
   static constexpr int kGroups = N / kCW;                  // softmax warpgroups
   static constexpr int kSoftWarps = 4 * kGroups;
-  static constexpr int kProdWarps = NB == 1 ? 4 : 2;   // gather issue rate scales with warps
+  // Two producer warps: with 19 warps per CTA no SM sub-partition (16K
+  // registers each) holds more than five, which leaves 96 registers per thread;
+  // a sixth warp on a sub-partition would cap every thread at 80 and spill
+  static constexpr int kProdWarps = 2;
   static constexpr int kThreads = 32 * (kSoftWarps + kProdWarps + 1);
   static constexpr int kStages = NB == 1 ? 4 : 2;
   static constexpr int kQBytes = N * kTcDim * 2;
   static constexpr int kKVBytes = kTcTile * kTcDim * 2;   // 32 KB
   static constexpr int kPBytes = kTcTile * N * 2;
-  // N = 64: the per-column row sums come from a second PV-shaped MMA with an
-  // all-ones A operand (L^T += 1 . P^T) into TMEM; N = 128 keeps them in registers
-  static constexpr bool kSumMma = NB == 1;
   // S^T and P^T buffers: three for N = 64, so QK runs two tiles ahead of the
   // softmax and ahead of the PV of the tile before (the tensor pipe executes in
   // issue order); two for N = 128 (TMEM is full)
   static constexpr int kSBuf = NB == 1 ? 3 : 2;
   static constexpr uint32_t kOCol = kSBuf * N;             // O^T x2 after the S buffers
-  static constexpr uint32_t kLCol = (kSBuf + 2) * N;       // L^T x2 (row-sum MMA)
-  static constexpr uint32_t kTmemCols = 512;               // 448 or 512 used
-  // all-ones A operand [128 x 16] in the no-swizzle K-major layout (8-row x
-  // 16-byte core matrices, 128 B apart along K, 256 B apart along M)
-  static constexpr int kOnesBytes = kSumMma ? 4096 : 1024;
+  static constexpr uint32_t kTmemCols = 512;               // 320 or 512 used
 };
 
 struct TcUnit {
@@ -107,7 +103,6 @@ struct __align__(1024) TcSmem {
   uint8_t q[2][C::kQBytes];
   uint8_t kv[C::kStages][C::kKVBytes];
   uint8_t p[C::kSBuf][C::kPBytes];
-  uint8_t ones[C::kOnesBytes];   // bf16 1.0 (A operand of the row-sum MMA)
   uint64_t kv_full[C::kStages], kv_empty[C::kStages];
   uint64_t q_full[2], q_empty[2], o_full[2], o_empty[2];
   uint64_t s_full[C::kSBuf], s_free[C::kSBuf], p_full[C::kSBuf], p_empty[C::kSBuf];
@@ -206,6 +201,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+// the two bf16 halves of a packed pair, widened exactly to fp32
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
   uint32_t r;
   asm volatile(
@@ -337,9 +335,6 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
   }
   for (int h = threadIdx.x; h < 128; h += blockDim.x)
     sm.sink_l2[h] = (args.sink != nullptr && h < args.Hq) ? args.sink[h] * 1.4426950408889634f : -INFINITY;
-  for (int o = threadIdx.x * 16; o < C::kOnesBytes; o += blockDim.x * 16)
-    *reinterpret_cast<uint4*>(sm.ones + o) = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-  fence_proxy_async();
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem, C::kTmemCols);
     tmem_relinquish();
@@ -352,7 +347,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
   if (warp >= kProd0 && warp < kMmaWarp) {
     // ===================================================================== producer
     const int pw = warp - kProd0;              // producer warp pw: tile rows [RW pw, RW pw + RW)
-    constexpr int RW = kTcTile / C::kProdWarps;        // 16 or 64 rows per warp
+    constexpr int RW = kTcTile / C::kProdWarps;        // 64 rows per warp
     constexpr int NI = (RW + 31) / 32;                  // 32-row index chunks per warp
     static_assert(RW % 32 == 0, "each producer warp owns whole 32-row index chunks");
     const int cbase = (RW * pw) / 32;                   // first 32-row chunk of this warp's rows
@@ -517,8 +512,6 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, N, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16(128, N, 1, 1);
-      constexpr uint32_t idesc_sum = idesc_bf16(128, N, 0, 1);
-      const uint32_t ones_base = smem_u32(sm.ones);
       int it = 0, kvc = 0, gt = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < args.n_units && ok; u += gridDim.x, ++it) {
@@ -568,12 +561,6 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           for (int j = 0; j < kTcTile / 16; ++j)
             mma_bf16(tmem + C::kOCol + ob * N, desc_mnmajor(kb, kTcTile * 128, j),
                      desc_mnmajor(pbase, kTcTile * 128, j), idesc_pv, (i > 0 || j > 0) ? 1u : 0u);
-          if constexpr (C::kSumMma) {
-#pragma unroll
-            for (int j = 0; j < kTcTile / 16; ++j)
-              mma_bf16(tmem + C::kLCol + ob * N, make_sdesc(ones_base, 128, 256, kLayoutNone),
-                       desc_mnmajor(pbase, kTcTile * 128, j), idesc_sum, (i > 0 || j > 0) ? 1u : 0u);
-          }
           tc_commit(&sm.kv_empty[stage]);
           tc_commit(&sm.p_empty[pb]);
         }
@@ -594,7 +581,6 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     const int col0 = CW * wg;
     const float sl2 = args.scale_log2;
-    constexpr bool kSumMma = C::kSumMma;
     int it = 0, gt = 0;
     for (int u = blockIdx.x; u < args.n_units; u += gridDim.x, ++it) {
       const int slot = it & 1;
@@ -603,9 +589,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       const int n_rows = inf.n_cp + inf.n_w;
       const int ob = it & 1, ouse = it >> 1;
       // running column maxima in registers (same in every thread of the
-      // warpgroup); per-thread row-sum partials unless the MMA keeps the sums
+      // warpgroup) and this thread's row-sum partials of its CW columns
       float mreg[CW];
-      float lpart[kSumMma ? 1 : CW];
+      float lpart[CW];
       // The running max starts at the head's sink logit: the sink is part of
       // every denominator, so m >= sigma is a valid stabiliser from the first
       // row on, and a unit's first tile needs no exact max unless a logit
@@ -619,7 +605,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         allset = allset && sg > -INFINITY;
       }
 #pragma unroll
-      for (int c = 0; c < (kSumMma ? 1 : CW); ++c) lpart[c] = 0.f;
+      for (int c = 0; c < CW; ++c) lpart[c] = 0.f;
       if (row < CW) {
         const float sg = sm.sink_l2[inf.hoff + ((col0 + row) & (args.H - 1))];
         sm.mcol[wg][row] = sg > -INFINITY ? sg : kNoRowMax;
@@ -700,14 +686,15 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           for (int c8 = 0; c8 < CW; c8 += 8) {
             float pv[8];
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              pv[e] = fast_ex2(s[c8 + e]);
-              pv[e + 1] = fast_ex2(s[c8 + e + 1]);
-              if constexpr (!kSumMma)
-                fadd2(lpart[(c8 + e) % (kSumMma ? 1 : CW)], lpart[(c8 + e + 1) % (kSumMma ? 1 : CW)], pv[e], pv[e + 1]);
-            }
+            for (int e = 0; e < 8; ++e) pv[e] = fast_ex2(s[c8 + e]);
             const uint32_t w0 = pack_bf16(pv[0], pv[1]), w1 = pack_bf16(pv[2], pv[3]);
             const uint32_t w2 = pack_bf16(pv[4], pv[5]), w3 = pack_bf16(pv[6], pv[7]);
+            // the row sums add the bf16-rounded weights that PV multiplies, so
+            // the normalisation matches the numerator term by term
+            fadd2(lpart[c8 + 0], lpart[c8 + 1], bf16_lo(w0), bf16_hi(w0));
+            fadd2(lpart[c8 + 2], lpart[c8 + 3], bf16_lo(w1), bf16_hi(w1));
+            fadd2(lpart[c8 + 4], lpart[c8 + 5], bf16_lo(w2), bf16_hi(w2));
+            fadd2(lpart[c8 + 6], lpart[c8 + 7], bf16_lo(w3), bf16_hi(w3));
             const int chunk = ((col0 & 63) >> 3) + (c8 >> 3);
             const uint32_t addr = prow + ((chunk ^ (row & 7)) << 4);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1), "r"(w2), "r"(w3)
@@ -776,25 +763,19 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
               break;
             }
             tc_fence_after();
+            const uint32_t oaddr = tmem + lane_addr + C::kOCol + ob * N + col0;
 #pragma unroll
-            for (int buf = 0; buf < (kSumMma ? 2 : 1); ++buf) {
-              // O^T, and with the row-sum MMA also L^T, share the column scaling
-              const uint32_t oaddr = tmem + lane_addr + (buf == 0 ? C::kOCol : C::kLCol) + ob * N + col0;
+            for (int h2 = 0; h2 < CW / 16; ++h2) {
+              uint32_t v[16];
+              tmem_ld16(oaddr + 16 * h2, v);
+              tmem_ld_wait();
 #pragma unroll
-              for (int h2 = 0; h2 < CW / 16; ++h2) {
-                uint32_t v[16];
-                tmem_ld16(oaddr + 16 * h2, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                  v[c] = __float_as_uint(__uint_as_float(v[c]) * sm.alpha[wg][16 * h2 + c]);
-                tmem_st16(oaddr + 16 * h2, v);
-              }
+              for (int c = 0; c < 16; ++c)
+                v[c] = __float_as_uint(__uint_as_float(v[c]) * sm.alpha[wg][16 * h2 + c]);
+              tmem_st16(oaddr + 16 * h2, v);
             }
-            if constexpr (!kSumMma) {
 #pragma unroll
-              for (int c = 0; c < (kSumMma ? 1 : CW); ++c) lpart[c] *= sm.alpha[wg][c];
-            }
+            for (int c = 0; c < CW; ++c) lpart[c] *= sm.alpha[wg][c];
             tmem_st_wait();
             tc_fence_before();
           }
@@ -807,57 +788,36 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       }
       if (!ok) break;
       if (threadIdx.x == 0) CSA_TR(it, 14, 0);
-      // ---- unit epilogue: per-column row sums l (TMEM L^T, or the 128 rows'
-      // partials: butterfly so lane l ends with column l's warp total, then the
-      // 4-warp total), output scale 2^(m-M) / (l 2^(m-M) + 2^(sigma-M)) with
-      // M = max(m, sigma), and lse (natural log, sink excluded)
-      if constexpr (!kSumMma) {
-        // butterfly over CW lanes: lane l ends with column l % CW summed over
-        // its CW-lane group; then add the 32 / CW groups
+      // ---- unit epilogue: per-column row sums l (butterfly so lane l ends
+      // with column l % CW summed over the warp's 32 rows, then the 4 warps
+      // through shared memory), output scale 2^(m-M) / (l 2^(m-M) + 2^(sigma-M))
+      // with M = max(m, sigma), and lse = (m + log2 l) ln 2 (sink excluded).
+      // None of it reads O^T, so it overlaps the unit's last PV.
 #pragma unroll
-        for (int st = CW / 2; st >= 1; st >>= 1) {
-          const bool up = (lane & st) != 0;
+      for (int st = CW / 2; st >= 1; st >>= 1) {
+        const bool up = (lane & st) != 0;
 #pragma unroll
-          for (int e = 0; e < st; ++e) {
-            const float send = up ? lpart[e % (kSumMma ? 1 : CW)] : lpart[(e + st) % (kSumMma ? 1 : CW)];
-            const float keep = up ? lpart[(e + st) % (kSumMma ? 1 : CW)] : lpart[e % (kSumMma ? 1 : CW)];
-            lpart[e % (kSumMma ? 1 : CW)] = keep + __shfl_xor_sync(0xffffffffu, send, st);
-          }
+        for (int e = 0; e < st; ++e) {
+          const float send = up ? lpart[e] : lpart[e + st];
+          const float keep = up ? lpart[e + st] : lpart[e];
+          lpart[e] = keep + __shfl_xor_sync(0xffffffffu, send, st);
         }
-#pragma unroll
-        for (int o = CW; o < 32; o <<= 1) lpart[0] += __shfl_xor_sync(0xffffffffu, lpart[0], o);
-        if (lane < CW) sm.xch[wg][wq][lane] = lpart[0];
-        named_bar_sync(bar_id, 128);
       }
-      if (!tc_wait(&sm.o_full[ob], ouse & 1, args.status, abort_flag)) break;
-      tc_fence_after();
-      if (threadIdx.x == 0) CSA_TR(it, 15, 6);
-      // Every thread derives its group's CW column scales itself: the column
-      // maxima are in mreg, and the row sums are in every lane of L^T (row-sum
-      // MMA) or in the butterfly totals.  scale = 2^(m-M) / (l 2^(m-M) +
-      // 2^(sigma-M)), M = max(m, sigma); lse = (m + log2 l) ln 2 (sink excluded).
-      float colv[CW];       // row sum, then output scale
-      if constexpr (kSumMma) {
-        uint32_t v[CW];
-        tmem_ld16(tmem + lane_addr + C::kLCol + ob * N + col0, v);
-        if constexpr (CW == 32) tmem_ld16(tmem + lane_addr + C::kLCol + ob * N + col0 + 16, v + 16);
-        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < CW; ++c) colv[c] = __uint_as_float(v[c]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < CW; ++c)
-          colv[c] = (sm.xch[wg][0][c] + sm.xch[wg][1][c]) + (sm.xch[wg][2][c] + sm.xch[wg][3][c]);
-      }
+      for (int o = CW; o < 32; o <<= 1) lpart[0] += __shfl_xor_sync(0xffffffffu, lpart[0], o);
+      if (lane < CW) sm.xch[wg][wq][lane] = lpart[0];
+      named_bar_sync(bar_id, 128);
       bool redo_local = tainted;
+      float colv[CW];       // output scales of the group's CW columns
       {
         // lane c (mod CW) of every warp computes column c once; the CW scales
-        // are then broadcast within the warp with shuffles (no shared memory)
+        // are then broadcast within the warp with shuffles
         const int c = lane % CW;
-        float l = 0.f, mcl = 0.f;
+        const float l = (sm.xch[wg][0][c] + sm.xch[wg][1][c]) + (sm.xch[wg][2][c] + sm.xch[wg][3][c]);
+        float mcl = 0.f;
 #pragma unroll
         for (int e = 0; e < CW; ++e)
-          if (e == c) { l = colv[e]; mcl = mreg[e]; }
+          if (e == c) mcl = mreg[e];
         const int col = col0 + c;
         const int h = inf.hoff + (col & (args.H - 1));
         const bool tok_ok = (col >> args.hshift) < inf.ntok;
@@ -883,6 +843,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       // group-wide decision; a tainted group recomputes its own columns exactly
       const bool redo = bar_red_or(bar_id, 128, redo_local);
       if (threadIdx.x == 0) CSA_TR(it, 14, 1);
+      if (!tc_wait(&sm.o_full[ob], ouse & 1, args.status, abort_flag)) break;
+      tc_fence_after();
+      if (threadIdx.x == 0) CSA_TR(it, 15, 6);
       if (redo) {
         tc_unit_exact(args, inf, sm.sink_l2, col0, col0 + CW, wq, 4);
       } else {
