@@ -68,7 +68,9 @@ struct TcCfg {
   static constexpr int kSoftWarps = 4 * kGroups;
   // Two producer warps: with 19 warps per CTA no SM sub-partition (16K
   // registers each) holds more than five, which leaves 96 registers per thread;
-  // a sixth warp on a sub-partition would cap every thread at 80 and spill
+  // a sixth warp on a sub-partition would cap every thread at 80 and spill.
+  // Two suffice for every tile kind: TMA loads contiguous tiles, and the
+  // per-row gathers use loops with little address arithmetic per row.
   static constexpr int kProdWarps = 2;
   static constexpr int kThreads = 32 * (kSoftWarps + kProdWarps + 1);
   static constexpr int kStages = NB == 1 ? 4 : 2;
@@ -464,8 +466,37 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
             cp_async16(dst, rb + static_cast<size_t>(s_g) * kTcDim, 16u);
           }
           cp_async_mbar_arrive(&sm.kv_full[stage]);
+        } else if (!args.sparse) {
+          // dense tile mixing entries, padding and window rows (or a tile the
+          // window wraps in): each instruction moves two 256-byte rows (lanes
+          // 0-15 / 16-31); the window's ring slots advance by one per row from
+          // the tile's first window row (one modulo per tile)
+          const int half = lane >> 4, c = lane & 15;
+          const int Lw0 = max(L0, n_cp);
+          const int sw0 = n_w > 0 ? (jlo + (Lw0 - n_cp)) % args.raw_cap : 0;
+          const __nv_bfloat16* kvb = args.kv_c + static_cast<size_t>(b) * args.kv_bstride * kTcDim + c * 8;
+          const __nv_bfloat16* rwb = args.kv_raw + static_cast<size_t>(b) * args.raw_cap * kTcDim + c * 8;
+#pragma unroll 8
+          for (int j = 0; j < RW / 2; ++j) {
+            const int rr = RW * pw + 2 * j + half;         // tile row
+            const int L = L0 + rr;
+            const __nv_bfloat16* src = kvb;
+            uint32_t bytes = 0;
+            if (L < n_c) {
+              src = kvb + static_cast<size_t>(L) * kTcDim;
+              bytes = 16;
+            } else if (L >= n_cp && L < n_rows) {
+              int slot = sw0 + (L - Lw0);                   // < 2 raw_cap: the window fits the ring
+              if (slot >= args.raw_cap) slot -= args.raw_cap;
+              src = rwb + static_cast<size_t>(slot) * kTcDim;
+              bytes = 16;
+            }
+            cp_async16(ks + sw128_off(rr, c, kTcTile), src, bytes);
+          }
+          cp_async_mbar_arrive(&sm.kv_full[stage]);
         } else {
-          // gather: each instruction moves two 256-byte rows (lanes 0-15 / 16-31)
+          // sparse tile past the selected entries: each instruction moves two
+          // 256-byte rows (lanes 0-15 / 16-31)
           int tr[NI];
 #pragma unroll
           for (int q = 0; q < NI; ++q) tr[q] = 0;
