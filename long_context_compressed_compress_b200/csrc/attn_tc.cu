@@ -619,9 +619,8 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       const TcUnit inf = sm.info[slot];
       const int n_rows = inf.n_cp + inf.n_w;
       const int ob = it & 1, ouse = it >> 1;
-      // running column maxima in registers (same in every thread of the
-      // warpgroup) and this thread's row-sum partials of its CW columns
-      float mreg[CW];
+      // this thread's row-sum partials of its CW columns; the running column
+      // maxima (the same for every thread of the warpgroup) live in sm.mcol
       float lpart[CW];
       // The running max starts at the head's sink logit: the sink is part of
       // every denominator, so m >= sigma is a valid stabiliser from the first
@@ -632,7 +631,6 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
 #pragma unroll
       for (int c = 0; c < CW; ++c) {
         const float sg = sm.sink_l2[inf.hoff + ((col0 + c) & (args.H - 1))];
-        mreg[c] = sg > -INFINITY ? sg : kNoRowMax;
         allset = allset && sg > -INFINITY;
       }
 #pragma unroll
@@ -695,14 +693,16 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         if (allset) {
 #pragma unroll
           for (int c = 0; c < CW; c += 2) {
-            ffma2(s[c], s[c + 1], s[c], s[c + 1], sl2, sl2, -mreg[c], -mreg[c + 1]);
+            const float2 m2 = *reinterpret_cast<const float2*>(&sm.mcol[wg][c]);
+            ffma2(s[c], s[c + 1], s[c], s[c + 1], sl2, sl2, -m2.x, -m2.y);
             dmax = fmaxf(dmax, fmaxf(s[c], s[c + 1]));
           }
         } else {
 #pragma unroll
           for (int c = 0; c < CW; ++c) {
-            const bool sen = mreg[c] == kNoRowMax;
-            s[c] = fmaf(s[c], sl2, sen ? 0.f : -mreg[c]);
+            const float mc = sm.mcol[wg][c];
+            const bool sen = mc == kNoRowMax;
+            s[c] = fmaf(s[c], sl2, sen ? 0.f : -mc);
             if (sen) newrow |= s[c] > -INFINITY;
             else dmax = fmaxf(dmax, s[c]);
           }
@@ -779,7 +779,6 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
             const float4 m4 = *reinterpret_cast<const float4*>(&sm.mcol[wg][c4]);
             const float4 d4 = *reinterpret_cast<const float4*>(&sm.dlt[wg][c4]);
             const float4 a4 = *reinterpret_cast<const float4*>(&sm.alpha[wg][c4]);
-            mreg[c4] = m4.x; mreg[c4 + 1] = m4.y; mreg[c4 + 2] = m4.z; mreg[c4 + 3] = m4.w;
             s[c4] -= d4.x; s[c4 + 1] -= d4.y; s[c4 + 2] -= d4.z; s[c4 + 3] -= d4.w;
             rescale |= (a4.x != 1.f) | (a4.y != 1.f) | (a4.z != 1.f) | (a4.w != 1.f);
             any_unset |= (m4.x == kNoRowMax) | (m4.y == kNoRowMax) | (m4.z == kNoRowMax) | (m4.w == kNoRowMax);
@@ -819,6 +818,10 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       }
       if (!ok) break;
       if (threadIdx.x == 0) CSA_TR(it, 14, 0);
+      // the unit's fields are read again here rather than kept in registers
+      // through the tile loop (the producer rewrites this slot only after the
+      // softmax warps release it below)
+      const TcUnit ue = sm.info[slot];
       // ---- unit epilogue: per-column row sums l (butterfly so lane l ends
       // with column l % CW summed over the warp's 32 rows, then the 4 warps
       // through shared memory), output scale 2^(m-M) / (l 2^(m-M) + 2^(sigma-M))
@@ -848,10 +851,10 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         float mcl = 0.f;
 #pragma unroll
         for (int e = 0; e < CW; ++e)
-          if (e == c) mcl = mreg[e];
+          if (e == c) mcl = sm.mcol[wg][e];
         const int col = col0 + c;
-        const int h = inf.hoff + (col & (args.H - 1));
-        const bool tok_ok = (col >> args.hshift) < inf.ntok;
+        const int h = ue.hoff + (col & (args.H - 1));
+        const bool tok_ok = (col >> args.hshift) < ue.ntok;
         float scale = 0.f, lse_v = -INFINITY;
         if (mcl > 0.5f * kNoRowMax) {
           // approximate ex2 / rcp / lg2 (relative error ~2^-22) are ample for a
@@ -864,9 +867,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           if (l > 0.f) lse_v = (mcl + fast_lg2(l)) * 0.6931471805599453f;
         }
         // every weight underflowed although the unit has rows: recompute
-        if (tok_ok && l == 0.f && inf.n_c + inf.n_w > 0) redo_local = true;
+        if (tok_ok && l == 0.f && ue.n_c + ue.n_w > 0) redo_local = true;
         if (wq == 0 && lane < CW && args.lse != nullptr && tok_ok)
-          args.lse[(static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0 + (col >> args.hshift)) * args.Hq + h] =
+          args.lse[(static_cast<size_t>(ue.b) * args.Tq + args.row0 + ue.r0 + (col >> args.hshift)) * args.Hq + h] =
               lse_v;
 #pragma unroll
         for (int e = 0; e < CW; ++e) colv[e] = __shfl_sync(0xffffffffu, scale, e);
@@ -878,7 +881,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       tc_fence_after();
       if (threadIdx.x == 0) CSA_TR(it, 15, 6);
       if (redo) {
-        tc_unit_exact(args, inf, sm.sink_l2, col0, col0 + CW, wq, 4);
+        tc_unit_exact(args, ue, sm.sink_l2, col0, col0 + CW, wq, 4);
       } else {
         const uint32_t oaddr = tmem + lane_addr + C::kOCol + ob * N + col0;
         const int d = row;
@@ -888,7 +891,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         tmem_ld_wait();
         if (threadIdx.x == 0) CSA_TR(it, 14, 2);
         __nv_bfloat16* obase =
-            args.out + ((static_cast<size_t>(inf.b) * args.Tq + args.row0 + inf.r0) * args.Hq + inf.hoff) * kTcDim + d;
+            args.out + ((static_cast<size_t>(ue.b) * args.Tq + args.row0 + ue.r0) * args.Hq + ue.hoff) * kTcDim + d;
         // lane pairs trade half their columns so that each lane holds two
         // adjacent head dims of CW/2 columns: the even lane columns [0, CW/2)
         // at dims (d, d + 1), the odd lane columns [CW/2, CW) at (d - 1, d);
@@ -904,7 +907,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           const int c = odd ? HC + j : j;
           const int col = col0 + c;
           const uint32_t w = odd ? pack_bf16(recv, hi) : pack_bf16(lo, recv);
-          if ((col >> args.hshift) < inf.ntok)
+          if ((col >> args.hshift) < ue.ntok)
             *reinterpret_cast<uint32_t*>(pbase + static_cast<size_t>(col) * kTcDim) = w;
         }
       }
