@@ -112,6 +112,7 @@ struct __align__(1024) TcSmem {
   float mcol[C::kGroups][C::kCW];
   float alpha[C::kGroups][C::kCW];
   float dlt[C::kGroups][C::kCW];
+  float oscale[C::kGroups][C::kCW];   // output scales of a unit whose read-out is pending
   float sink_l2[128];      // sink logits in log2 units (-inf without a sink)
   TcUnit info[2];
   uint32_t tmem;
@@ -613,6 +614,44 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
     const int col0 = CW * wg;
     const float sl2 = args.scale_log2;
     int it = 0, gt = 0;
+    // A unit's O^T read-out is deferred until the next unit's first tile is
+    // done, so the wait for its last PV overlaps useful work: the group's
+    // column scales wait in sm.oscale, and these registers hold the rest.
+    bool pend = false;
+    int pend_ob = 0;
+    uint32_t pend_par = 0, pend_cols = 0;   // o_full parity; columns with a token
+    __nv_bfloat16* pend_out = nullptr;      // head dim `row` of the unit's first output row
+    auto flush = [&]() -> bool {
+      if (!tc_wait(&sm.o_full[pend_ob], pend_par, args.status, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t oaddr = tmem + lane_addr + C::kOCol + pend_ob * N + col0;
+      uint32_t v[CW];
+      tmem_ld16(oaddr, v);
+      if constexpr (CW == 32) tmem_ld16(oaddr + 16, v + 16);
+      tmem_ld_wait();
+      if (threadIdx.x == 0) CSA_TR(it, 14, 2);
+      // lane pairs trade half their columns so that each lane holds two
+      // adjacent head dims of CW/2 columns: the even lane columns [0, CW/2)
+      // at dims (d, d + 1), the odd lane columns [CW/2, CW) at (d - 1, d);
+      // then one 4-byte bf16x2 store per column
+      constexpr int HC = CW / 2;
+      const bool odd = (lane & 1) != 0;
+      __nv_bfloat16* pbase = pend_out - (odd ? 1 : 0);
+#pragma unroll
+      for (int j = 0; j < HC; ++j) {
+        const float lo = __uint_as_float(v[j]) * sm.oscale[wg][j];
+        const float hi = __uint_as_float(v[HC + j]) * sm.oscale[wg][HC + j];
+        const float recv = __shfl_xor_sync(0xffffffffu, odd ? lo : hi, 1);
+        const int c = odd ? HC + j : j;
+        const uint32_t w = odd ? pack_bf16(recv, hi) : pack_bf16(lo, recv);
+        if ((pend_cols >> c) & 1u)
+          *reinterpret_cast<uint32_t*>(pbase + static_cast<size_t>(col0 + c) * kTcDim) = w;
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.o_empty[pend_ob]);
+      pend = false;
+      return true;
+    };
     for (int u = blockIdx.x; u < args.n_units; u += gridDim.x, ++it) {
       const int slot = it & 1;
       if (!tc_wait(&sm.q_full[slot], (it >> 1) & 1, args.status, abort_flag)) break;
@@ -815,6 +854,10 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         fence_proxy_async();
         mbar_arrive(&sm.p_full[pb]);
         if (threadIdx.x == 0) CSA_TR(it, i, 5);
+        if (i == 0 && pend && !flush()) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) break;
       if (threadIdx.x == 0) CSA_TR(it, 14, 0);
@@ -842,10 +885,9 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
       if (lane < CW) sm.xch[wg][wq][lane] = lpart[0];
       named_bar_sync(bar_id, 128);
       bool redo_local = tainted;
-      float colv[CW];       // output scales of the group's CW columns
       {
-        // lane c (mod CW) of every warp computes column c once; the CW scales
-        // are then broadcast within the warp with shuffles
+        // lane c (mod CW) of every warp computes column c once; warp 0 keeps
+        // the CW scales in sm.oscale for the read-out
         const int c = lane % CW;
         const float l = (sm.xch[wg][0][c] + sm.xch[wg][1][c]) + (sm.xch[wg][2][c] + sm.xch[wg][3][c]);
         float mcl = 0.f;
@@ -871,53 +913,33 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
         if (wq == 0 && lane < CW && args.lse != nullptr && tok_ok)
           args.lse[(static_cast<size_t>(ue.b) * args.Tq + args.row0 + ue.r0 + (col >> args.hshift)) * args.Hq + h] =
               lse_v;
-#pragma unroll
-        for (int e = 0; e < CW; ++e) colv[e] = __shfl_sync(0xffffffffu, scale, e);
+        if (wq == 0 && lane < CW) sm.oscale[wg][lane] = scale;
       }
       // group-wide decision; a tainted group recomputes its own columns exactly
       const bool redo = bar_red_or(bar_id, 128, redo_local);
       if (threadIdx.x == 0) CSA_TR(it, 14, 1);
-      if (!tc_wait(&sm.o_full[ob], ouse & 1, args.status, abort_flag)) break;
-      tc_fence_after();
-      if (threadIdx.x == 0) CSA_TR(it, 15, 6);
       if (redo) {
+        if (!tc_wait(&sm.o_full[ob], ouse & 1, args.status, abort_flag)) break;
+        tc_fence_after();
         tc_unit_exact(args, ue, sm.sink_l2, col0, col0 + CW, wq, 4);
+        tc_fence_before();
+        mbar_arrive(&sm.o_empty[ob]);
       } else {
-        const uint32_t oaddr = tmem + lane_addr + C::kOCol + ob * N + col0;
-        const int d = row;
-        uint32_t v[CW];
-        tmem_ld16(oaddr, v);
-        if constexpr (CW == 32) tmem_ld16(oaddr + 16, v + 16);
-        tmem_ld_wait();
-        if (threadIdx.x == 0) CSA_TR(it, 14, 2);
-        __nv_bfloat16* obase =
-            args.out + ((static_cast<size_t>(ue.b) * args.Tq + args.row0 + ue.r0) * args.Hq + ue.hoff) * kTcDim + d;
-        // lane pairs trade half their columns so that each lane holds two
-        // adjacent head dims of CW/2 columns: the even lane columns [0, CW/2)
-        // at dims (d, d + 1), the odd lane columns [CW/2, CW) at (d - 1, d);
-        // then one 4-byte bf16x2 store per column
-        constexpr int HC = CW / 2;
-        const bool odd = (lane & 1) != 0;
-        __nv_bfloat16* pbase = obase - (odd ? 1 : 0);
+        pend = true;
+        pend_ob = ob;
+        pend_par = static_cast<uint32_t>(ouse & 1);
+        pend_out = args.out + ((static_cast<size_t>(ue.b) * args.Tq + args.row0 + ue.r0) * args.Hq + ue.hoff) * kTcDim + row;
+        uint32_t cols = 0;
 #pragma unroll
-        for (int j = 0; j < HC; ++j) {
-          const float lo = __uint_as_float(v[j]) * colv[j];
-          const float hi = __uint_as_float(v[HC + j]) * colv[HC + j];
-          const float recv = __shfl_xor_sync(0xffffffffu, odd ? lo : hi, 1);
-          const int c = odd ? HC + j : j;
-          const int col = col0 + c;
-          const uint32_t w = odd ? pack_bf16(recv, hi) : pack_bf16(lo, recv);
-          if ((col >> args.hshift) < ue.ntok)
-            *reinterpret_cast<uint32_t*>(pbase + static_cast<size_t>(col) * kTcDim) = w;
-        }
+        for (int c = 0; c < CW; ++c)
+          if (((col0 + c) >> args.hshift) < ue.ntok) cols |= 1u << c;
+        pend_cols = cols;
       }
-      if (threadIdx.x == 0) CSA_TR(it, 14, 3);
-      tc_fence_before();
-      mbar_arrive(&sm.o_empty[ob]);
       if (threadIdx.x == 0) CSA_TR(it, 15, 7);
-      named_bar_sync(bar_id, 128);      // mcol / alpha reused by the next unit
+      named_bar_sync(bar_id, 128);      // mcol / alpha reused, oscale visible to the group
       mbar_arrive(&sm.q_empty[slot]);
     }
+    if (pend) flush();
   }
   tc_fence_before();
   __syncthreads();
