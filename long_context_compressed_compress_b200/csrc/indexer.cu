@@ -30,12 +30,23 @@ template <int NQ> struct IdxShape {
   static constexpr int tiles = NQ > 16 ? 8 : 16;
   static constexpr int stages = NQ > 16 ? 2 : 4;
 };
-// TMEM columns: accumulator NQ + SFA 4 + SFB 4, rounded to a power of two
-template <int NQ> struct IdxTmem { static constexpr uint32_t cols = NQ + 8 <= 32 ? 32 : (NQ + 8 <= 128 ? 128 : 256); };
+// The narrow tile double-buffers its accumulator (the MMA of tile j+1 runs
+// during the epilogue of tile j); the wide one cannot without halving the
+// CTAs that share an SM's TMEM.
+template <int NQ> struct IdxAcc { static constexpr int bufs = NQ <= 16 ? 2 : 1; };
+// TMEM columns: accumulators and key scales (SFA, 4 columns) bufs times each,
+// query scales (SFB) 4, rounded to a power of two
+template <int NQ> struct IdxTmem {
+  static constexpr int used = IdxAcc<NQ>::bufs * (NQ + 4) + 4;
+  static constexpr uint32_t cols = used <= 32 ? 32 : (used <= 64 ? 64 : (used <= 128 ? 128 : 256));
+};
 // shared-memory floor per CTA so that no more CTAs share an SM than its 512
 // TMEM columns hold (a CTA waiting in tcgen05.alloc would only idle)
 template <int NQ> struct IdxFloor {
-  static constexpr size_t bytes = IdxTmem<NQ>::cols == 256 ? 96 * 1024 : (IdxTmem<NQ>::cols == 128 ? 48 * 1024 : 0);
+  static constexpr size_t bytes = IdxTmem<NQ>::cols == 256   ? 96 * 1024
+                                  : IdxTmem<NQ>::cols == 128 ? 48 * 1024
+                                  : IdxTmem<NQ>::cols == 64  ? 27 * 1024
+                                                             : 0;
 };
 
 template <int NS>
@@ -45,7 +56,7 @@ struct __align__(128) IdxSmem {
   uint8_t sfa[NS][512];
   uint8_t sfb[512];
   float w[128];
-  uint64_t mbar;
+  uint64_t mbar[2];
   uint32_t tmem;
   int abort_flag;
 };
@@ -95,7 +106,8 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&sm.mbar, 1);
+    mbar_init(&sm.mbar[0], 1);
+    mbar_init(&sm.mbar[1], 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -150,32 +162,66 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
-  const uint32_t t_acc = tmem, t_sfa = tmem + NQ, t_sfb = tmem + NQ + 4;
+  constexpr int NB = IdxAcc<NQ>::bufs;
+  // per buffer b: accumulator at b NQ, key scales at NB NQ + 4 b; query scales last
+  const uint32_t t_sfa0 = tmem + NB * NQ, t_sfb = tmem + NB * NQ + 4 * NB;
   constexpr uint32_t idesc = idesc_nvfp4(128, NQ);
   const uint64_t bdesc = make_sdesc(smem_u32(sm.qB), 128, 256, kLayoutNone);
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-
-  for (int j = 0; j < ntiles; ++j) {
-    const int stage = j % NS;
-    cp_async_wait<NS - 1>();
-    fence_proxy_async();
-    __syncthreads();
-    if (sm.abort_flag) break;
+  // the narrow tile keeps its NQ folded weights in registers
+  float wr[NQ <= 16 ? NQ : 1];
+  if constexpr (NQ <= 16) {
+#pragma unroll
+    for (int c = 0; c < NQ; ++c) wr[c] = sm.w[c];
+  }
+  // MMA of tile j (thread 0): scales to TMEM, block-scaled FP4 MMA, commit
+  auto issue_mma = [&](int j) {
     if (tid == 0) {
       tc_fence_after();
       if (j == 0) tmem_cp_32x128b_x4(t_sfb, make_sdesc(smem_u32(sm.sfb), 128, 128, kLayoutNone));
+      const int stage = j % NS;
+      const uint32_t t_sfa = t_sfa0 + 4 * (j % NB);
       tmem_cp_32x128b_x4(t_sfa, make_sdesc(smem_u32(sm.sfa[stage]), 128, 128, kLayoutNone));
       const uint64_t adesc = make_sdesc(smem_u32(sm.kA[stage]), 128, 256, kLayoutNone);
-      mma_nvfp4(t_acc, adesc, bdesc, idesc, t_sfa, t_sfb, 0u);
-      tc_commit(&sm.mbar);
+      mma_nvfp4(tmem + (j % NB) * NQ, adesc, bdesc, idesc, t_sfa, t_sfb, 0u);
+      tc_commit(&sm.mbar[j % NB]);
     }
-    if (!mbar_wait(&sm.mbar, static_cast<uint32_t>(j & 1), status)) sm.abort_flag = 1;
+  };
+  if constexpr (NB == 2) {
+    cp_async_wait<NS - 1>();
+    fence_proxy_async();
+    __syncthreads();
+    issue_mma(0);
+  }
+
+  for (int j = 0; j < ntiles; ++j) {
+    const int stage = j % NS;
+    if constexpr (NB == 2) {
+      // tile j+1's keys are in (groups 0 .. j+1 of NS + j committed); its MMA
+      // goes into the other accumulator, whose epilogue (tile j-1) is done
+      if (j + 1 < ntiles) {
+        cp_async_wait<NS - 2>();
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        if (sm.abort_flag) break;
+        issue_mma(j + 1);
+      }
+    } else {
+      cp_async_wait<NS - 1>();
+      fence_proxy_async();
+      __syncthreads();
+      if (sm.abort_flag) break;
+      issue_mma(j);
+    }
+    if (!mbar_wait(&sm.mbar[j % NB], static_cast<uint32_t>((j / NB) & 1), status)) sm.abort_flag = 1;
     tc_fence_after();
     // the MMA has consumed this stage: prefetch NS tiles ahead into it
     if (j + NS < ntiles) load_k_tile(et0 + j + NS, stage);
     cp_async_commit();
 
     // ---- epilogue: this thread owns entry s; columns are (token, head) pairs
+    const uint32_t t_acc = tmem + (j % NB) * NQ;
     const int s = (et0 + j) * 128 + tid;
     const bool s_ok = s < S;
     constexpr int CB = NQ % 32 == 0 ? 32 : 16;   // columns per TMEM load
@@ -188,12 +234,17 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
 #pragma unroll
       for (int tt = 0; tt < CB / HI; ++tt) {
         const int t = c0 / HI + tt;
+        if constexpr (NQ <= 16) {
+          if (t >= ntok) break;   // uniform: a decode chunk fills few of the tile's tokens
+        }
         float acc = 0.f;
 #pragma unroll
-        for (int h = 0; h < HI; ++h)
-          acc = fmaf(sm.w[c0 + tt * HI + h], fmaxf(__uint_as_float(v[tt * HI + h]), 0.f), acc);
+        for (int h = 0; h < HI; ++h) {
+          const float wv = NQ <= 16 ? wr[(tt * HI + h) % (NQ <= 16 ? NQ : 1)] : sm.w[c0 + tt * HI + h];
+          acc = fmaf(wv, fmaxf(__uint_as_float(v[tt * HI + h]), 0.f), acc);
+        }
         const long long p = pbase + t;
-        if (s_ok && t < ntok && static_cast<long long>(m) * (s + 1) - 1 <= p)
+        if (s_ok && (NQ <= 16 || t < ntok) && static_cast<long long>(m) * (s + 1) - 1 <= p)
           score[(static_cast<size_t>(bi) * T_chunk + tq0 + t) * ld + s] = static_cast<TS>(acc);
       }
     }

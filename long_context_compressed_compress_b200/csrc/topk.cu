@@ -789,7 +789,7 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_count(const __nv_bfloat16*
   }
 }
 
-__global__ void __launch_bounds__(kMcThreads) topk_mc_emit(const __nv_bfloat16* __restrict__ score, int T_chunk,
+__global__ void __launch_bounds__(kMcThreads, 4) topk_mc_emit(const __nv_bfloat16* __restrict__ score, int T_chunk,
                                                            int S, int ld, int k, int m, int row0,
                                                            const int32_t* __restrict__ q_pos0,
                                                            const int* __restrict__ ws, int32_t* __restrict__ idx) {
@@ -821,7 +821,8 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_emit(const __nv_bfloat16* 
   const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
   const bool al = (reinterpret_cast<uintptr_t>(srow) & 15) == 0;
   const int r0 = i0 + kMcRun * threadIdx.x;
-  uint32_t kr[kMcRun];
+  // the run's 16-bit keys, two per register (key q in half q & 1 of kr[q / 2])
+  uint32_t kr[kMcRun / 2];
 #pragma unroll
   for (int gq = 0; gq < kMcRun / 8; ++gq) {
     uint32_t kk[8];
@@ -833,13 +834,14 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_emit(const __nv_bfloat16* 
       for (int q = 0; q < 8; ++q) kk[q] = 0u;
     }
 #pragma unroll
-    for (int q = 0; q < 8; ++q) kr[8 * gq + q] = kk[q];
+    for (int q = 0; q < 8; q += 2) kr[4 * gq + q / 2] = kk[q] | (kk[q + 1] << 16);
   }
+  auto key_at = [&](int q) -> uint32_t { return (kr[q >> 1] >> (16 * (q & 1))) & 0xFFFFu; };
   int n_gt = 0, n_eq = 0;
 #pragma unroll
   for (int q = 0; q < kMcRun; ++q) {
-    n_gt += r0 + q < i1 && kr[q] > K;
-    n_eq += r0 + q < i1 && kr[q] == K;
+    n_gt += r0 + q < i1 && key_at(q) > K;
+    n_eq += r0 + q < i1 && key_at(q) == K;
   }
   int tg, te;
   const int gt_t = block_excl_scan_nt<kMcThreads>(n_gt, wsum, &tg);
@@ -849,9 +851,10 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_emit(const __nv_bfloat16* 
   for (int q = 0; q < kMcRun; ++q) {
     const int i = r0 + q;
     if (i < i1) {
-      if (kr[q] > K) {
+      const uint32_t key = key_at(q);
+      if (key > K) {
         out[pos++] = i;
-      } else if (kr[q] == K) {
+      } else if (key == K) {
         if (eq_seen < krem) out[pos++] = i;
         ++eq_seen;
       }
