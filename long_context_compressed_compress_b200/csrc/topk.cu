@@ -575,14 +575,16 @@ int launch_topk_run(const T* score, long long rows, int T_chunk, int S, int ld, 
 // ---------------------------------------------------------------------------
 // Multi-CTA select for a few long BF16 rows (decode: 32 rows of 262144 scores).
 // A row is cut into chunks of kMcChunk keys, one CTA per (row, chunk), and the
-// radix select runs as four launches that meet through a caller workspace:
+// radix select runs as three launches that meet through a caller workspace:
 //   K1  11-bit histogram of the high key bits      -> ws hist1[row][2048]
 //   K2  threshold bin b1 (every CTA scans hist1),
 //       5-bit histogram of the keys in bin b1       -> ws hist2[row][32]
-//   K3  exact threshold key K and the count krem of keys == K to take;
-//       per-chunk counts of keys > K and == K       -> ws cnt[row][chunk][2]
-//   K4  in-order compaction: the chunk's output offset is the sum over earlier
-//       chunks, then per-warp segments with ballots, as in the one-CTA kernel.
+//       and per chunk: its keys above bin b1 and its own 5-bit histogram of
+//       bin b1                                     -> ws chunk[row][c][33]
+//   K3  exact threshold key K = (b1, b2) and the count krem of keys == K to
+//       take (every CTA scans hist2); the counts of keys > K and == K in the
+//       earlier chunks follow from their K2 records, which give the chunk's
+//       output offset; then in-order compaction over per-thread runs.
 // The histograms are cleared by a memset at the start of every call.  The
 // union of per-chunk results is the exact row result with the same tie rule.
 // ---------------------------------------------------------------------------
@@ -597,9 +599,13 @@ constexpr int kMcMinS = 16384;      // shorter rows use one CTA per row
 struct McLayout {
   int C;            // chunks per row
   size_t row_ints;  // ints per row
-  // per row: hist1[2048] hist2[32] state[4] cnt[C][2]
+  // per row: hist1[2048] hist2[32] state[4] chunk[C][1 + 32] (keys above bin
+  // b1, then the chunk's 5-bit histogram of bin b1)
   static constexpr int kHist2 = kMcHist1, kState = kMcHist1 + kMcHist2, kCnt = kMcHist1 + kMcHist2 + 4;
-  __host__ __device__ McLayout(int S) : C((S + kMcChunk - 1) / kMcChunk), row_ints(kCnt + 2 * static_cast<size_t>((S + kMcChunk - 1) / kMcChunk)) {}
+  static constexpr int kChunkInts = 1 + kMcHist2;
+  __host__ __device__ McLayout(int S)
+      : C((S + kMcChunk - 1) / kMcChunk),
+        row_ints(kCnt + kChunkInts * static_cast<size_t>((S + kMcChunk - 1) / kMcChunk)) {}
 };
 
 __device__ __forceinline__ int mc_row_n(int row, int T_chunk, int S, int m, int row0, const int32_t* q_pos0) {
@@ -719,50 +725,7 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_hist2(const __nv_bfloat16*
   const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
   const bool al = (reinterpret_cast<uintptr_t>(srow) & 15) == 0;
   const int r0 = i0 + kMcRun * threadIdx.x;
-#pragma unroll
-  for (int g = 0; g < kMcRun / 8; ++g) {
-    const int b = r0 + 8 * g;
-    if (b < i1) {
-      uint32_t kk[8];
-      mc_load8(srow, b, i1, ld, al, kk);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (b + q < i1 && static_cast<int>(kk[q] >> 5) == b1) atomicAdd(&h2[kk[q] & 31], 1);
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x < kMcHist2 && h2[threadIdx.x]) atomicAdd(&g[McLayout::kHist2 + threadIdx.x], h2[threadIdx.x]);
-}
-
-__global__ void __launch_bounds__(kMcThreads) topk_mc_count(const __nv_bfloat16* __restrict__ score, int T_chunk,
-                                                            int S, int ld, int k, int m, int row0,
-                                                            const int32_t* __restrict__ q_pos0, int* __restrict__ ws) {
-  using KO = KeyOf<__nv_bfloat16>;
-  __shared__ int h2[kMcHist2];
-  __shared__ int wsum[kMcWarps];
-  __shared__ int s_bin, s_above;
-  __shared__ int wc[kMcWarps][2];
-  const McLayout L(S);
-  const int row = blockIdx.x / L.C, c = blockIdx.x % L.C;
-  const int n = mc_row_n(row, T_chunk, S, m, row0, q_pos0);
-  if (n <= k) return;
-  int* g = ws + static_cast<size_t>(row) * L.row_ints;
-  if (threadIdx.x < kMcHist2) h2[threadIdx.x] = g[McLayout::kHist2 + threadIdx.x];
-  __syncthreads();
-  const int b1 = g[McLayout::kState + 0];
-  const int krem1 = k - g[McLayout::kState + 1];
-  mc_find_bin<kMcHist2>(h2, krem1, wsum, &s_bin, &s_above);
-  const uint32_t K = (static_cast<uint32_t>(b1) << 5) | static_cast<uint32_t>(s_bin);
-  const int krem = krem1 - s_above;
-  if (c == 0 && threadIdx.x == 0) {
-    g[McLayout::kState + 2] = static_cast<int>(K);
-    g[McLayout::kState + 3] = krem;
-  }
-  const int i0 = c * kMcChunk, i1 = min(n, i0 + kMcChunk);
-  const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
-  const bool al = (reinterpret_cast<uintptr_t>(srow) & 15) == 0;
-  const int r0 = i0 + kMcRun * threadIdx.x;
-  int n_gt = 0, n_eq = 0;
+  int n_above = 0;   // this thread's keys above bin b1
 #pragma unroll
   for (int g = 0; g < kMcRun / 8; ++g) {
     const int b = r0 + 8 * g;
@@ -771,21 +734,28 @@ __global__ void __launch_bounds__(kMcThreads) topk_mc_count(const __nv_bfloat16*
       mc_load8(srow, b, i1, ld, al, kk);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        n_gt += b + q < i1 && kk[q] > K;
-        n_eq += b + q < i1 && kk[q] == K;
+        const int bin = static_cast<int>(kk[q] >> 5);
+        if (b + q < i1) {
+          n_above += bin > b1;
+          if (bin == b1) atomicAdd(&h2[kk[q] & 31], 1);
+        }
       }
     }
   }
-  n_gt = __reduce_add_sync(0xffffffffu, n_gt);
-  n_eq = __reduce_add_sync(0xffffffffu, n_eq);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (lane == 0) { wc[warp][0] = n_gt; wc[warp][1] = n_eq; }
+  n_above = __reduce_add_sync(0xffffffffu, n_above);
+  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = n_above;
   __syncthreads();
+  int* rec = g + McLayout::kCnt + static_cast<size_t>(c) * McLayout::kChunkInts;
+  if (threadIdx.x < kMcHist2) {
+    const int v = h2[threadIdx.x];
+    rec[1 + threadIdx.x] = v;
+    if (v) atomicAdd(&g[McLayout::kHist2 + threadIdx.x], v);
+  }
   if (threadIdx.x == 0) {
-    int a = 0, b = 0;
-    for (int w = 0; w < kMcWarps; ++w) { a += wc[w][0]; b += wc[w][1]; }
-    g[McLayout::kCnt + 2 * c] = a;
-    g[McLayout::kCnt + 2 * c + 1] = b;
+    int a = 0;
+#pragma unroll
+    for (int w = 0; w < kMcWarps; ++w) a += wsum[w];
+    rec[0] = a;
   }
 }
 
@@ -794,6 +764,8 @@ __global__ void __launch_bounds__(kMcThreads, 4) topk_mc_emit(const __nv_bfloat1
                                                            const int32_t* __restrict__ q_pos0,
                                                            const int* __restrict__ ws, int32_t* __restrict__ idx) {
   __shared__ int wsum[kMcWarps];
+  __shared__ int h2s[kMcHist2];
+  __shared__ int s_bin, s_above, s_gt, s_eq;
   const McLayout L(S);
   const int row = blockIdx.x / L.C, c = blockIdx.x % L.C;
   const int n = mc_row_n(row, T_chunk, S, m, row0, q_pos0);
@@ -808,14 +780,34 @@ __global__ void __launch_bounds__(kMcThreads, 4) topk_mc_emit(const __nv_bfloat1
   const int i1 = min(n, i0 + kMcChunk);
   if (i0 >= i1) return;
   const int* g = ws + static_cast<size_t>(row) * L.row_ints;
-  const uint32_t K = static_cast<uint32_t>(g[McLayout::kState + 2]);
-  const int krem = g[McLayout::kState + 3];
-  // keys > K and == K in the chunks before this one
-  int gt_c = 0, eq_c = 0;
-  for (int cc = 0; cc < c; ++cc) {
-    gt_c += g[McLayout::kCnt + 2 * cc];
-    eq_c += g[McLayout::kCnt + 2 * cc + 1];
+  // threshold K = (b1, b2): b2 from the row's 5-bit histogram of bin b1
+  if (threadIdx.x < kMcHist2) h2s[threadIdx.x] = g[McLayout::kHist2 + threadIdx.x];
+  __syncthreads();
+  const int b1 = g[McLayout::kState + 0];
+  const int krem1 = k - g[McLayout::kState + 1];
+  mc_find_bin<kMcHist2>(h2s, krem1, wsum, &s_bin, &s_above);
+  const int b2 = s_bin;
+  const uint32_t K = (static_cast<uint32_t>(b1) << 5) | static_cast<uint32_t>(b2);
+  const int krem = krem1 - s_above;
+  // keys > K and == K in the chunks before this one (lane l sums chunks l, l + 32, ...)
+  if (threadIdx.x < 32) {
+    int gt = 0, eq = 0;
+    for (int cc = threadIdx.x; cc < c; cc += 32) {
+      const int* rec = g + McLayout::kCnt + static_cast<size_t>(cc) * McLayout::kChunkInts;
+      int a = rec[0];
+      for (int bb = b2 + 1; bb < kMcHist2; ++bb) a += rec[1 + bb];
+      gt += a;
+      eq += rec[1 + b2];
+    }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    eq = __reduce_add_sync(0xffffffffu, eq);
+    if (threadIdx.x == 0) {
+      s_gt = gt;
+      s_eq = eq;
+    }
   }
+  __syncthreads();
+  const int gt_c = s_gt, eq_c = s_eq;
   // this thread's run, then its output position: every key > K before it in
   // the row, plus the keys == K before it that are taken (the first krem)
   const __nv_bfloat16* srow = score + static_cast<size_t>(row) * ld;
@@ -878,7 +870,6 @@ int launch_topk_multi(const __nv_bfloat16* score, long long rows, int T_chunk, i
   const unsigned grid = static_cast<unsigned>(rows * L.C);
   topk_mc_hist1<<<grid, kMcThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, ws);
   topk_mc_hist2<<<grid, kMcThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, ws);
-  topk_mc_count<<<grid, kMcThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, ws);
   topk_mc_emit<<<grid, kMcThreads, 0, st>>>(score, T_chunk, S, ld, k, m, row0, q_pos0, ws, idx);
   return check_launch();
 }

@@ -172,7 +172,8 @@ class CsaDecode:
         nws = ops.topk_workspace_size(B, 1, cap, c.k)
         self.ws = torch.empty((max(1, nws // 4),), dtype=torch.int32, device=device) if nws else None
         self.sink = state.get("sink")
-        self.launches = 6 + 2 + 1 + 1 + 1 + (5 if nws else 1) + 1 + 1
+        # multi-CTA top-k: workspace memset + three kernels
+        self.launches = 6 + 2 + 1 + 1 + 1 + (4 if nws else 1) + 1 + 1
         self.graph = None
         self.x = None
 
