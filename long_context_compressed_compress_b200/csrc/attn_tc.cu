@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
           // dense tile mixing entries, padding and window rows (or a tile the
           // window wraps in): each instruction moves two 256-byte rows (lanes
           // 0-15 / 16-31); the window's ring slots advance by one per row from
-          // the tile's first window row (one modulo per tile)
+          // the tile's first window row (one modulo per tile, then wrap-arounds)
           const int half = lane >> 4, c = lane & 15;
           const int Lw0 = max(L0, n_cp);
           const int sw0 = n_w > 0 ? (jlo + (Lw0 - n_cp)) % args.raw_cap : 0;
@@ -487,8 +487,10 @@ __global__ void __launch_bounds__(TcCfg<NB>::kThreads, 1) attn_tc_kernel(const T
               src = kvb + static_cast<size_t>(L) * kTcDim;
               bytes = 16;
             } else if (L >= n_cp && L < n_rows) {
-              int slot = sw0 + (L - Lw0);                   // < 2 raw_cap: the window fits the ring
-              if (slot >= args.raw_cap) slot -= args.raw_cap;
+              // the unit's window (W + G - 1 rows for G tokens) may exceed the
+              // ring, so the slot can pass raw_cap more than once
+              int slot = sw0 + (L - Lw0);
+              while (slot >= args.raw_cap) slot -= args.raw_cap;
               src = rwb + static_cast<size_t>(slot) * kTcDim;
               bytes = 16;
             }

@@ -417,6 +417,27 @@ def test_ring_window_decode_positions(ops):
     _attn_tol("bf16")(_np(out), oracle.round_out(ro, "bf16"))
 
 
+@pytest.mark.parametrize("H,cap", [(16, 128), (16, 130), (32, 129), (64, 128), (128, 200)])
+def test_hca_dense_ring_window(ops, H, cap):
+    """Dense (HCA) calls with a raw ring (raw_cap < T): the window reads slot
+    j % raw_cap, also when a unit of G = 64/H tokens spans W + G - 1 positions,
+    more than the ring holds (the slot wraps more than once within a tile)."""
+    B, D, W, m, T = 2, 128, 128, 16, 6
+    p0 = np.array([3001, 777])
+    S = int(p0.max() + T) // m + 4
+    q = _randn((B, T, H, D), "bf16", 80)
+    kv_c = _randn((B, S, D), "bf16", 81)
+    ring = _randn((B, cap, D), "bf16", 82)
+    sink = torch.randn((H,), generator=torch.Generator().manual_seed(83))
+    out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device="cuda")
+    pos0 = torch.from_numpy(p0.astype(np.int32)).cuda()
+    ops.hca_dense_attn_fwd(q.cuda(), kv_c.cuda(), ring.cuda(), sink.cuda(), 1 / np.sqrt(D), W, pos0, out, m,
+                           raw_cap=cap)
+    pos = p0[:, None] + np.arange(T)[None]
+    ro, _ = oracle.dense_attn(q, kv_c, ring, cap, sink, 1 / np.sqrt(D), W, pos, m)
+    _attn_tol("bf16")(_np(out), oracle.round_out(ro, "bf16"))
+
+
 def test_attn_rescale_path(ops):
     """Later KV tiles with far larger logits force the running-max rescale of the
     O^T accumulator and row sums (tiles ordered: entries, then the window)."""
