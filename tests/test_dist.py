@@ -59,3 +59,26 @@ def test_reference_arm_is_rank0_only(capsys):
         steps, warmup, gpus, T = 1, 0, 2, 0
     assert bench.run_reference(A(), configs.CSA_PREFILL, rank=1) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank0(capsys):
+    """Rank 0 times the oracle on a bounded sample and prints one JSON line with
+    the contract's keys (impl, metric/value/unit, cpu_baseline, zero-byte e2e)."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    from long_context_compressed_compress_b200 import configs
+
+    class A:
+        steps, warmup, gpus, T = 1, 0, 1, 512
+    bench.run_reference(A(), configs.scaled(configs.CSA_PREFILL, T=512), rank=0)
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["T"] == 512
