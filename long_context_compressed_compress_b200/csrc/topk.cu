@@ -203,12 +203,16 @@ __global__ void __launch_bounds__(kTopkThreads) topk_row_kernel(const T* __restr
 // shared offset t Lp, with Lp / V odd (V keys per 16-byte vector): the 16-byte
 // reads of a quarter-warp then fall in distinct bank groups.  The first digit's
 // histogram is taken while the row is loaded; each later digit re-reads the
-// runs.  Histogram atomics go to kRunCopies copies picked by lane, so lanes
-// whose keys share a bin (scores crowd into a few exponents) rarely collide.
+// runs.  Histogram atomics go to RunCopies<NT>::n copies picked by lane, so
+// lanes whose keys share a bin (scores crowd into a few exponents) rarely collide.
 // Compaction: per-thread counts of keys > K and == K, two block scans for the
 // output offsets, then every thread writes its own selections in index order.
 // ---------------------------------------------------------------------------
-constexpr int kRunCopies = 8;
+// Histogram copies per block size.  128-thread rows (up to 16K keys) trade
+// atomic collisions for occupancy: fewer copies leave shared memory for more
+// CTAs per SM (2 copies: 0.34 ms against 0.39 ms with 8 on the 32K-token
+// prefill rows).  512-thread rows run one CTA per SM and keep 8.
+template <int NT> struct RunCopies { static constexpr int n = NT <= 128 ? 2 : 8; };
 
 template <int NT>
 __device__ __forceinline__ int block_excl_scan_nt(int v, int* wsum, int* total) {
@@ -244,12 +248,12 @@ __device__ __forceinline__ void block_select16(const uint32_t (&kk)[MAXP], int c
                                                int* sel_digit, int* sel_above, uint32_t* K_out, int* krem_out) {
   constexpr int DPT = (256 + NT - 1) / NT;
   const int tid = threadIdx.x;
-  const int cp = tid & (kRunCopies - 1);
+  const int cp = tid & (RunCopies<NT>::n - 1);
   uint32_t prefix = 0, pmask = 0;
   int krem = r;
 #pragma unroll 1
   for (int shift = 8; shift >= 0; shift -= 8) {
-    for (int i = tid; i < kRunCopies * 256; i += NT) hflat[i] = 0;
+    for (int i = tid; i < RunCopies<NT>::n * 256; i += NT) hflat[i] = 0;
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < MAXP; ++q)
@@ -262,7 +266,7 @@ __device__ __forceinline__ void block_select16(const uint32_t (&kk)[MAXP], int c
       int c = 0;
       if (d >= 0) {
 #pragma unroll
-        for (int c2 = 0; c2 < kRunCopies; ++c2) c += hflat[c2 * 256 + d];
+        for (int c2 = 0; c2 < RunCopies<NT>::n; ++c2) c += hflat[c2 * 256 + d];
       }
       cq[q] = c;
       csum += c;
@@ -299,7 +303,7 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
   constexpr int DPT = (256 + NT - 1) / NT;
   constexpr int top = KO::bits - 8;
   extern __shared__ __align__(16) uint8_t dsm[];
-  __shared__ int hist[kRunCopies][256];
+  __shared__ int hist[RunCopies<NT>::n][256];
   __shared__ int wsum[NT / 32];
   __shared__ int sel_digit, sel_above;
 
@@ -320,8 +324,8 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
   run_shape<NT, V>(n, &L, &Lp);
   K* keys = reinterpret_cast<K*>(dsm);
   int* hflat = &hist[0][0];
-  const int cp = lane & (kRunCopies - 1);
-  for (int i = tid; i < kRunCopies * 256; i += NT) hflat[i] = 0;
+  const int cp = lane & (RunCopies<NT>::n - 1);
+  for (int i = tid; i < RunCopies<NT>::n * 256; i += NT) hflat[i] = 0;
   __syncthreads();
 
   // rows that try the sampled threshold first take their first-digit
@@ -448,7 +452,7 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
         return;
       }
       // fall back to the full radix path: take its first-digit histogram now
-      for (int i = tid; i < kRunCopies * 256; i += NT) hflat[i] = 0;
+      for (int i = tid; i < RunCopies<NT>::n * 256; i += NT) hflat[i] = 0;
       __syncthreads();
       for (int j = 0; j < cnt; j += V) {
         const uint4 u = *reinterpret_cast<const uint4*>(run + j);
@@ -465,7 +469,7 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
 #pragma unroll 1
   for (int shift = top; shift >= 0; shift -= 8) {
     if (shift != top) {
-      for (int i = tid; i < kRunCopies * 256; i += NT) hflat[i] = 0;
+      for (int i = tid; i < RunCopies<NT>::n * 256; i += NT) hflat[i] = 0;
       __syncthreads();
       for (int j = 0; j < cnt; j += V) {
         const uint4 u = *reinterpret_cast<const uint4*>(run + j);
@@ -486,7 +490,7 @@ __global__ void __launch_bounds__(NT) topk_run_kernel(const T* __restrict__ scor
       int c = 0;
       if (d >= 0) {
 #pragma unroll
-        for (int c2 = 0; c2 < kRunCopies; ++c2) c += hist[c2][d];
+        for (int c2 = 0; c2 < RunCopies<NT>::n; ++c2) c += hist[c2][d];
       }
       cq[q] = c;
       csum += c;
