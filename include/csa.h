@@ -186,7 +186,9 @@ size_t topk_workspace_size(int B, int T_chunk, int S, int k);
  *   - concurrency: calls that overlap in time on the same device (other
  *     streams, other host threads) share that scratch and race; order them.
  *   - set-up: the first call on a device (with that device current) looks up
- *     the scratch address; make it before any stream capture begins.
+ *     the scratch address; make it before any stream capture begins.  The
+ *     address is kept for the life of the process, so after cudaDeviceReset
+ *     this entry must not be called on that device again.
  */
 int topk_select_noalloc(const void* score, int score_dtype, int B, int T_chunk,
                         int S, int score_ld, int k, int m, int row0,

@@ -945,13 +945,15 @@ int topk_select(const void* score, int score_dtype, int B, int T_chunk, int S, i
 // Limits and rules, in plain words:
 //   * the scratch holds kNoAllocScratchBytes (1 MiB); a shape whose multi-CTA
 //     histograms need more is rejected with CSA_ERR_UNSUPPORTED before any
-//     work is queued (32 rows of 262,144 entries need about 275 KB);
+//     work is queued (32 rows of 262,144 entries need about 402 KB);
 //   * the scratch is one per device and per process: two calls that overlap
 //     in time on the same device (different streams, or different host
 //     threads) race on it and give wrong results;
 //   * the first call on each device looks up the scratch's device address
 //     (cudaGetSymbolAddress with that device current); make that first call
-//     before any stream capture begins;
+//     before any stream capture begins.  The address is cached for the life
+//     of the process: after cudaDeviceReset the cached address is stale, so
+//     a caller that resets a device must not call this entry on it again;
 //   * shapes that need no scratch run the one-CTA-per-row kernel, as
 //     topk_select does without a workspace.
 // ---------------------------------------------------------------------------

@@ -430,6 +430,12 @@ def csa_decode_step(st, x, p, m, k, W, tau, dtype, gscale=1.0):
         prev = slice(((i + 1) % 2) * m, ((i + 1) % 2) * m + m)
 
         def entry(a, b, z):
+            # entry 0 has no predecessor block: its softmax covers the m current
+            # logits only, exactly as in prefill ([cf-1] §3.1 overlap needs a
+            # previous block; the first block has none)
+            if i == 0:
+                cur_rows = [st["carry_" + n][:, cur] for n in (a, b, z)]
+                return round_out(csa_compress(cur_rows[0], cur_rows[1], cur_rows[2], m), dtype)
             slab = [np.concatenate([st["carry_" + n][:, prev], st["carry_" + n][:, cur]], axis=1) for n in (a, b, z)]
             return round_out(csa_compress(slab[0], slab[1], slab[2], m, first_has_pred=True), dtype)
 

@@ -138,3 +138,11 @@ def test_decode_full_size_sampled(L):
     the GPU runs all sequences; the oracle checks sequences 0, 13 and 31 over
     four steps (the fourth emits an entry)."""
     run_decode(L, configs.CSA_DECODE, [0, 13, 31], 4, graph=False)
+
+
+def test_decode_from_empty_cache(L):
+    """Twelve steps from position 0 with an empty cache: the window is partly
+    empty, no entry is visible before p = 3, and p = 3 emits entry 0, whose
+    softmax covers only its own block's m logits (no predecessor)."""
+    cfg = dataclasses.replace(configs.CSA_DECODE, B=3, T0=0, steps=12)
+    run_decode(L, cfg, [0, 1, 2], 12, graph=False)

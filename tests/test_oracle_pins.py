@@ -397,31 +397,64 @@ def test_bf16_rounding_matches_torch_on_fp32_inputs():
     np.testing.assert_array_equal(formats.bf16(x.astype(np.float64)), ref)
 
 
-def test_decode_steps_equal_prefill_rows():
-    """Decoding token p from a cache built from tokens [0, T0) gives row p of a
-    prefill over the same tokens: pins the decode step's carry slots, emission
-    timing (entry (p+1)/m - 1 visible at step p), NVFP4 keys and ring window."""
+def _decode_from(T0, T=96, W=16):
+    """Decode tokens T0..T-1 from a cache built from tokens [0, T0) and return
+    (per-step results, full prefill oracle result, final state)."""
     from long_context_compressed_compress_b200 import configs, inputs
-    cfg = configs.scaled(configs.PR1, T=96, k=8)
-    m, W, T0 = cfg.m, 16, 64
+    cfg = configs.scaled(configs.PR1, T=T, k=8)
+    m = cfg.m
     x = inputs.layer_inputs(cfg, device="cpu")
     full = oracle.csa_layer(x, m, cfg.k, W, cfg.tau, cfg.dtype)
     f = {k: v.to(torch.float64).numpy() for k, v in x.items()}
     st = {"kv_c": oracle.round_out(oracle.csa_compress(f["a"][:, :T0], f["b"][:, :T0], f["z"][:, :T0], m), "f32"),
           "ring": np.zeros((cfg.B, W, cfg.D))}
     k_src = oracle.round_out(oracle.csa_compress(f["a_I"][:, :T0], f["b_I"][:, :T0], f["z_I"][:, :T0], m), "f32")
-    st["khat"] = oracle.nvfp4_quantize(k_src)["xhat"]
-    for j in range(T0 - W, T0):
+    st["khat"] = oracle.nvfp4_quantize(k_src)["xhat"] if k_src.shape[1] else np.zeros((cfg.B, 0, cfg.DI))
+    for j in range(max(0, T0 - W), T0):
         st["ring"][:, j % W] = f["kv_raw"][:, j]
+    # the carry holds the raw rows of the last complete block and of the
+    # block in progress
     for n in ("a", "b", "z", "a_I", "b_I", "z_I"):
         c = np.zeros((cfg.B, 2 * m, f[n].shape[-1]))
-        for j in range(T0 - m, T0):
+        for j in range(max(0, (T0 // m - 1) * m), T0):
             c[:, j % (2 * m)] = f[n][:, j]
         st["carry_" + n] = c
+    res = []
     for p in range(T0, cfg.T):
         xs = {n: f[n][:, p] for n in ("q", "q_I", "w", "a", "b", "z", "a_I", "b_I", "z_I", "kv_raw")}
         xs["sink"] = f["sink"]
-        r = oracle.csa_decode_step(st, xs, p, m, cfg.k, W, cfg.tau, cfg.dtype)
+        res.append(oracle.csa_decode_step(st, xs, p, m, cfg.k, W, cfg.tau, cfg.dtype))
+    return res, full, st, cfg
+
+
+@pytest.mark.parametrize("T0", [64, 0, 1, 3, 5])
+def test_decode_steps_equal_prefill_rows(T0):
+    """Decoding token p from a cache built from tokens [0, T0) gives row p of a
+    prefill over the same tokens: pins the decode step's carry slots, emission
+    timing (entry (p+1)/m - 1 visible at step p), entry 0 without a predecessor
+    (T0 < m: the first block's softmax covers its own m logits only), NVFP4
+    keys and the ring window."""
+    res, full, st, cfg = _decode_from(T0)
+    for p, r in zip(range(T0, cfg.T), res):
         np.testing.assert_array_equal(r["idx"][0], full["idx"][p])     # rows are (b, t), B = 1
         np.testing.assert_allclose(r["out"][0], full["out"][p], rtol=1e-12, atol=1e-12)
-    assert st["kv_c"].shape[1] == cfg.T // m
+    assert st["kv_c"].shape[1] == cfg.T // cfg.m
+    # the emitted cache itself equals the prefill compressor's entries, entry 0
+    # included (a planted predecessor at entry 0 changes it: see the next test)
+    from long_context_compressed_compress_b200 import inputs
+    x = inputs.layer_inputs(cfg, device="cpu")
+    ref = oracle.round_out(oracle.csa_compress(x["a"], x["b"], x["z"], cfg.m), "f32")
+    np.testing.assert_array_equal(st["kv_c"], ref)
+
+
+def test_decode_entry0_differs_from_a_zero_predecessor():
+    """Entry 0 with a zero predecessor slab (8 logits, four of them 0) is not
+    entry 0 of the definition; the decode step must emit the latter."""
+    res, full, st, cfg = _decode_from(0, T=8)
+    f = {}
+    from long_context_compressed_compress_b200 import inputs
+    x = inputs.layer_inputs(cfg, device="cpu")
+    m = cfg.m
+    slab = [np.concatenate([np.zeros((1, m, cfg.D)), x[n][:, :m].double().numpy()], axis=1) for n in ("a", "b", "z")]
+    wrong = oracle.round_out(oracle.csa_compress(slab[0], slab[1], slab[2], m, first_has_pred=True), "f32")
+    assert np.abs(wrong[:, 0] - st["kv_c"][:, 0]).max() > 1e-3
