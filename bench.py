@@ -13,6 +13,16 @@ One JSON line on rank 0:
   kernels    per-kernel average duration (ms) and algorithmic rate
   cpu_baseline  the CPU oracle on a bounded sample of the same workload
 
+The default run also measures the two other throughputs the metric names and
+reports them under "workloads" in the same line, each with its own roofline,
+e2e, clocks and CPU baseline:
+  csa_decode_32x1m    decode steps/s: 32 sequences x 1,048,576 cached tokens,
+                      128 heads, top-k 1024, one new token per sequence per
+                      step, replayed from a CUDA graph
+  hca_prefill_2x128k  HCA prefill tokens/s: B = 2, T = 131072, 64 heads,
+                      ratio 128 (1024 entries per sequence), window + sink
+Each is also a line of its own with --workload.
+
 --impl reference times the CPU oracle as the reference arm (rank 0 only).
 Multi-GPU (torchrun): every rank runs its own independent layer (weak scaling,
 no collective on the data path; the timing uses a MAX all-reduce).
@@ -48,9 +58,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=0,
                     help="profiling case: override the layer's token count (not a bench line)")
-    ap.add_argument("--workload", default="csa_prefill_32k", choices=["csa_prefill_32k", "csa_decode_32x1m", "stack_hhcc_256k"],
-                    help="csa_prefill_32k (the default line), csa_decode_32x1m (decode steps/s) or "
-                         "stack_hhcc_256k (4-layer prefill stack tokens/s)")
+    ap.add_argument("--workload", default="csa_prefill_32k",
+                    choices=["csa_prefill_32k", "csa_decode_32x1m", "hca_prefill_2x128k", "stack_hhcc_256k"],
+                    help="csa_prefill_32k (the default line), csa_decode_32x1m (decode steps/s), "
+                         "hca_prefill_2x128k (HCA prefill tokens/s) or stack_hhcc_256k (4-layer prefill stack)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="default run only: skip the decode and HCA measurements under 'workloads'")
     return ap.parse_args()
 
 
@@ -195,11 +208,34 @@ class OracleSample:
         per_row = self.t_rows / max(1, self.n_rows)
         return self.cfg.B * self.cfg.T / (self.t_comp + per_row * self.cfg.B * self.cfg.T)
 
-    def describe(self):
-        return {"value": self.value(), "unit": "tokens/s", "cores": self.cores, "kind": "oracle",
-                "sample": f"compressors + NVFP4 over all {self.cfg.T} tokens ({self.t_comp:.1f} s), then "
-                          f"indexer/top-k/attention on {self.n_rows} uniform query rows "
-                          f"({self.t_rows:.1f} s), extrapolated to {self.cfg.T} rows"}
+    def single_thread(self, n_rows):
+        """The same sample on one host thread (numpy's pools limited to 1):
+        compressors again, then ``n_rows`` query rows; tokens/s."""
+        try:
+            from threadpoolctl import threadpool_limits
+        except ImportError:  # pragma: no cover
+            return None
+        o, c, x = self.oracle, self.cfg, self.x
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            o.csa_compress(x["a"], x["b"], x["z"], c.m)
+            o.nvfp4_quantize(o.round_out(o.csa_compress(x["a_I"], x["b_I"], x["z_I"], c.m), c.dtype))
+            t_comp = time.perf_counter() - t0
+            keep = (self.t_rows, self.n_rows)
+            self.t_rows, self.n_rows = 0.0, 0
+            self.rows(n_rows)
+            per_row = self.t_rows / max(1, self.n_rows)
+            self.t_rows, self.n_rows = keep
+        return c.B * c.T / (t_comp + per_row * c.B * c.T)
+
+    def describe(self, one_thread=None):
+        d = {"value": self.value(), "unit": "tokens/s", "cores": self.cores, "kind": "oracle",
+             "sample": f"compressors + NVFP4 over all {self.cfg.T} tokens ({self.t_comp:.1f} s), then "
+                       f"indexer/top-k/attention on {self.n_rows} uniform query rows "
+                       f"({self.t_rows:.1f} s), extrapolated to {self.cfg.T} rows"}
+        if one_thread is not None:
+            d["value_1thread"] = one_thread
+        return d
 
 
 def torch_f64():
@@ -210,7 +246,7 @@ def torch_f64():
 def cpu_baseline(cfg, n_rows):
     s = OracleSample(cfg)
     s.rows(n_rows)
-    return s.describe()
+    return s.describe(one_thread=s.single_thread(max(64, n_rows // 16)))
 
 
 def run_reference(args, cfg, rank):
@@ -263,6 +299,9 @@ def main():
         cfg = configs.scaled(cfg, T=args.T)
     if args.workload == "csa_decode_32x1m":
         main_decode(args, rank, world, local)
+        return
+    if args.workload == "hca_prefill_2x128k":
+        main_hca(args, rank, world, local)
         return
     if args.workload == "stack_hhcc_256k":
         main_stack(args, rank, world, local)
@@ -426,6 +465,19 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_rows)
+    if not args.no_extra and not args.T:
+        # the metric's other two throughputs, measured in the same run (every
+        # rank runs them, in the same order, as independent replicas)
+        del x, xd, host, lay
+        torch.cuda.empty_cache()
+        extra = {}
+        for name, fn in (("csa_decode_32x1m", measure_decode), ("hca_prefill_2x128k", measure_hca)):
+            sub = fn(args, rank, world, dev)
+            torch.cuda.empty_cache()
+            extra[name] = {k: sub[k] for k in ("value", "unit", "ms_per_step", "steps", "warmup", "config",
+                                               "roofline", "kernels", "e2e", "gpu_launches", "clocks",
+                                               "cpu_baseline") if k in sub}
+        line["workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -460,21 +512,28 @@ def decode_cpu_baseline(cfg, n_seq=2):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:  # pragma: no cover
         cores = 1
-    return {"value": 1.0 / (dt * cfg.B / n_seq), "unit": "steps/s", "cores": cores, "kind": "oracle",
-            "sample": f"one decode step for {n_seq} of the {cfg.B} sequences ({dt:.1f} s), "
-                      f"extrapolated to all {cfg.B}"}
+    d = {"value": 1.0 / (dt * cfg.B / n_seq), "unit": "steps/s", "cores": cores, "kind": "oracle",
+         "sample": f"one decode step for {n_seq} of the {cfg.B} sequences ({dt:.1f} s), "
+                   f"extrapolated to all {cfg.B}"}
+    try:
+        from threadpoolctl import threadpool_limits
+        o1 = {k: (v[:1].copy() if isinstance(v, np.ndarray) and v.ndim >= 2 else v) for k, v in o.items()}
+        x1 = {k: (v[:1] if k != "sink" else v) for k, v in x.items()}
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            oracle.csa_decode_step(o1, x1, cfg.T0, cfg.m, cfg.k, cfg.W, cfg.tau, cfg.dtype)
+            d["value_1thread"] = 1.0 / ((time.perf_counter() - t0) * cfg.B)
+    except ImportError:  # pragma: no cover
+        pass
+    return d
 
 
 def main_decode(args, rank, world, local):
-    """CSA decode at 1M context: B = 32 sequences x 1,048,576 cached tokens
-    (262,144 entries), H = 128, k = 1024; one step = one new token for every
-    sequence, replayed from a CUDA graph.  value = steps/s of the whole job."""
-    import dataclasses
+    """CSA decode at 1M context as a line of its own (see ``measure_decode``)."""
     import torch
     import torch.distributed as dist
     from long_context_compressed_compress_b200 import build, configs
     build.build()
-    from long_context_compressed_compress_b200 import inputs, layer
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if args.impl == "reference":
@@ -490,8 +549,26 @@ def main_decode(args, rank, world, local):
         return
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    line = measure_decode(args, rank, world, dev)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_decode(args, rank, world, dev):
+    """CSA decode at 1M context: B = 32 sequences x 1,048,576 cached tokens
+    (262,144 entries), H = 128, k = 1024; one step = one new token for every
+    sequence, replayed from a CUDA graph.  value = steps/s of the whole job.
+    At least 64 steps are timed (a multiple of m = 4, so entry emission is
+    amortised as in the workload's definition)."""
+    import dataclasses
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import configs, inputs, layer
+    steps = max(64, args.steps)
     n_kern = 8
-    total = args.warmup + args.steps + 2 * (args.e2e_steps + 2) + n_kern + 8
+    total = args.warmup + steps + 2 * (args.e2e_steps + 2) + n_kern + 8
     cfg = dataclasses.replace(configs.CSA_DECODE, steps=total)
     peaks = load_peaks()
     st = inputs.decode_state(cfg, device="cuda")
@@ -521,7 +598,7 @@ def main_decode(args, rank, world, local):
         lay.replay()
     torch.cuda.synchronize()
     props = torch.cuda.get_device_properties(dev)
-    sampler = ClockSampler("GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(local))
+    sampler = ClockSampler("GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(dev.index))
     sampler.start()
     if world > 1:
         dist.barrier()
@@ -530,7 +607,7 @@ def main_decode(args, rank, world, local):
     s0 = torch.cuda.Event(enable_timing=True)
     s1 = torch.cuda.Event(enable_timing=True)
     s0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         lay.replay()
     s1.record(stream)
     torch.cuda.synchronize()
@@ -541,7 +618,7 @@ def main_decode(args, rank, world, local):
     ms = s0.elapsed_time(s1)
     if world > 1:
         ms = max_over_ranks(ms, dev)
-    ms_step = ms / args.steps
+    ms_step = ms / steps
     # end to end: pinned host inputs copied in, the graph, the output read back
     host = {k: v.cpu().pin_memory() for k, v in x.items()}
     out_host = torch.empty(lay.out.shape, dtype=lay.out.dtype).pin_memory()
@@ -584,7 +661,7 @@ def main_decode(args, rank, world, local):
     achieved = idx_bytes / (it * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": world / (ms_step * 1e-3), "unit": "steps/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic cache drawn on the device (N(0,1) entries and indexer keys, seeded)",
         "config": {"workload": "csa_decode_32x1m", "B": B, "T0": cfg.T0, "S0": cfg.S0, "H": cfg.H, "D": cfg.D,
@@ -593,7 +670,7 @@ def main_decode(args, rank, world, local):
                    "l2": "inputs larger than L2 (302 MB of NVFP4 keys and 2.1 GB of KV per step's cache)"},
         "e2e": {"value": job_throughput(world, 1, e2e_ms), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms} if args.e2e_steps > 0 else None,
-        "gpu_launches": lay.launches * args.steps,
+        "gpu_launches": lay.launches * steps,
         "roofline": {"bound": "hbm", "kernel": "indexer_score", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": f"{peaks['source']} hbm_gbs", "algorithmic_bytes_per_launch": idx_bytes},
@@ -601,11 +678,198 @@ def main_decode(args, rank, world, local):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = decode_cpu_baseline(configs.CSA_DECODE)
+    lay.graph = None
+    return line
+
+
+def hca_cpu_baseline(cfg, x, n_rows=64, one_thread=True):
+    """The oracle's HCA layer on the host cores: the 128:1 compression of every
+    token, then dense attention for ``n_rows`` uniform query rows (seed 1234),
+    extrapolated to all B*T rows; the inputs are the device draw copied to the
+    host (outside the timed part), q only for the sampled rows."""
+    import numpy as np
+    import oracle
+    import torch
+
+    def run(rows_per_seq):
+        rng = np.random.default_rng(1234)
+        f = lambda t: t.to("cpu", torch.float64).numpy()
+        host = [(f(x["a"][b]), f(x["z"][b]), f(x["kv_raw"][b])) for b in range(cfg.B)]
+        ts = [np.sort(rng.integers(0, cfg.T, size=rows_per_seq)) for _ in range(cfg.B)]
+        qs = [f(x["q"][b, torch.from_numpy(t).to(x["q"].device)]) for b, t in enumerate(ts)]
+        sink = f(x["sink"])
+        t0 = time.perf_counter()
+        kvs = [oracle.round_out(oracle.hca_compress(a, z, cfg.m), cfg.dtype) for (a, z, _) in host]
+        t_comp = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        for b in range(cfg.B):
+            n = len(ts[b])
+            oracle.dense_attn(qs[b][None], kvs[b][None], host[b][2][None], cfg.T, sink, cfg.tau, cfg.W,
+                              ts[b][None], cfg.m, rows=[(0, i) for i in range(n)])
+        t_rows = time.perf_counter() - t0
+        n_tot = cfg.B * rows_per_seq
+        return cfg.B * cfg.T / (t_comp + t_rows / n_tot * cfg.B * cfg.T), t_comp, t_rows, n_tot
+
+    v, t_comp, t_rows, n_tot = run(max(1, n_rows // cfg.B))
+    try:
+        from threadpoolctl import threadpool_info, threadpool_limits
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        threadpool_limits, cores = None, 1
+    d = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+         "sample": f"128:1 compression of all {cfg.B}x{cfg.T} tokens ({t_comp:.1f} s), then dense attention "
+                   f"for {n_tot} uniform query rows ({t_rows:.1f} s), extrapolated to {cfg.B * cfg.T} rows"}
+    if one_thread and threadpool_limits is not None:
+        with threadpool_limits(limits=1):
+            d["value_1thread"] = run(max(1, n_rows // (4 * cfg.B)))[0]
+    return d
+
+
+def main_hca(args, rank, world, local):
+    """HCA prefill as a line of its own (see ``measure_hca``)."""
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import build, configs, inputs
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if args.impl == "reference":
+        if rank == 0:
+            cfg = configs.HCA_PREFILL
+            x = inputs.layer_inputs(cfg, device="cuda")
+            cb = hca_cpu_baseline(cfg, x, one_thread=False)
+            print(json.dumps({"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
+                              "n_gpus": args.gpus, "steps": 1, "warmup": 0, "higher_is_better": True,
+                              "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                              "config": {"workload": "hca_prefill_2x128k"}, "cpu_baseline": cb,
+                              "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    line = measure_hca(args, rank, world, dev)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    lay.graph = None
     if world > 1:
         dist.destroy_process_group()
+
+
+def measure_hca(args, rank, world, dev):
+    """HCA prefill: B = 2, T = 131072, 64 heads x dim 128, ratio 128 (1024
+    entries per sequence), window 128 + sink, gate logits N(0, 2); one step =
+    hca_compress + hca_dense_attn_fwd on inputs resident in HBM.  value = B*T
+    tokens per step time, whole job."""
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import configs, inputs, layer
+    cfg = configs.HCA_PREFILL
+    peaks = load_peaks()
+    x = inputs.layer_inputs(cfg, device="cuda")
+    lay = layer.HcaPrefill(cfg)
+    stream = torch.cuda.current_stream()
+    ev = {}
+
+    @contextlib.contextmanager
+    def timer(name):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        yield
+        e1.record(stream)
+        ev.setdefault(name, []).append((e0, e1))
+
+    steps = max(3, min(args.steps, 40))
+    for _ in range(args.warmup):
+        lay.run(x)
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid) if hasattr(props, "uuid") else str(dev.index))
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(steps):
+        lay.run(x, timer=timer)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    ms = s0.elapsed_time(s1)
+    if world > 1:
+        ms = max_over_ranks(ms, dev)
+    ms_step = ms / steps
+    kern = {k: sum(a.elapsed_time(b) for a, b in v) / steps for k, v in ev.items()}
+    flops = attn_flops(cfg)
+    comp_bytes = cfg.B * (2 * cfg.T * cfg.D * 2 + cfg.S * cfg.D * 2)
+    kernels = {}
+    for name, t in kern.items():
+        if name == "hca_dense_attn_fwd":
+            rate = flops / (t * 1e-3) / 1e12
+            kernels[name] = {"ms": round(t, 4), "achieved": round(rate, 1), "unit": "TFLOP/s",
+                             "frac": round(rate / peaks["bf16_tflops"], 4)}
+        else:
+            rate = comp_bytes / (t * 1e-3) / 1e9
+            kernels[name] = {"ms": round(t, 4), "achieved": round(rate, 1), "unit": "GB/s",
+                             "frac": round(rate / peaks["hbm_gbs"], 4)}
+    achieved = flops / (kern["hca_dense_attn_fwd"] * 1e-3) / 1e12
+    # end to end: pinned host inputs in, the layer, the output back
+    n_e2e = max(1, min(args.e2e_steps, 2)) if args.e2e_steps > 0 else 0
+    e2e = None
+    if n_e2e:
+        host = {k: v.cpu().pin_memory() for k, v in x.items()}
+        out_host = torch.empty(lay.out.shape, dtype=lay.out.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+
+        def e2e_step():
+            for k, v in host.items():
+                x[k].copy_(v, non_blocking=True)
+            lay.run(x)
+            out_host.copy_(lay.out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            e2e_ms = max_over_ranks(e2e_ms, dev)
+        e2e = {"value": job_throughput(world, cfg.B * cfg.T, e2e_ms), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        del host, out_host
+    line = {
+        "metric": METRIC, "value": job_throughput(world, cfg.B * cfg.T, ms_step), "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded inputs drawn on the device: a N(0,1), z N(0,2), q, kv_raw, sink N(0,1))",
+        "config": {"workload": "hca_prefill_2x128k", "B": cfg.B, "T": cfg.T, "H": cfg.H, "D": cfg.D, "m": cfg.m,
+                   "S": cfg.S, "W": cfg.W, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (q + out = 8.6 GB per step)"},
+        "e2e": e2e,
+        "gpu_launches": lay.launches * steps,
+        "roofline": {"bound": "tensor", "kernel": "hca_dense_attn_fwd", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": None, "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                     "algorithmic_flops_per_launch": flops},
+        "kernels": kernels, "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = hca_cpu_baseline(cfg, x)
+    del x, lay
+    return line
 
 
 def attn_flops(cfg):

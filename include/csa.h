@@ -67,10 +67,19 @@ const char* csa_status_string(int status);
 int csa_last_cuda_error(void);
 /* Library version as major*10000 + minor*100 + patch. */
 int csa_version(void);
-/* Synchronising read-and-clear of the device status word that kernels set
- * (instead of trapping) when a bounded wait gives up: CSA_OK or
- * CSA_ERR_TIMEOUT.  Returns CSA_ERR_CUDA if the copy fails. */
+/* Device status words.  Kernels that wait on other warps of their CTA
+ * (indexer_score, sparse_attn_fwd, hca_dense_attn_fwd) bound every wait in
+ * wall time; a wait that gives up makes the kernel skip its remaining work and
+ * return (it never traps) and stores CSA_ERR_TIMEOUT | (site << 8) into a
+ * status word: the int32 `status` the call was given (device memory owned by
+ * the caller, which sets it to 0 beforehand; the first failure is kept), or,
+ * when the call passed NULL, the library's per-device word.
+ * csa_device_status: synchronising read-and-clear of that per-device word
+ * (CSA_OK or CSA_ERR_TIMEOUT | site << 8); CSA_ERR_CUDA if the copy fails. */
 int csa_device_status(int* status_out);
+/* Wall-time limit of every bounded device wait, in nanoseconds, for kernels
+ * launched after the call (process-wide; 0 restores the default of 2 s). */
+int csa_set_wait_timeout_ns(uint64_t ns);
 
 /*
  * csa_compress -- gated overlapping m:1 KV compressor ([cf-1] §3.1: every 4
@@ -140,14 +149,14 @@ int nvfp4_quantize(const void* x, int in_dtype, int64_t rows, int D, float gscal
  *   positions q_pos0[b] + row0 + r.  Only visible (r, s) pairs are written.
  * Requires DI in {32, 64}, HI in {1, 2, 4, 8}, score_ld >= S; q_fp4 and k_fp4
  * 16-byte aligned, and k_sf 4-byte aligned when DI = 64 (else
- * CSA_ERR_ALIGNMENT).
+ * CSA_ERR_ALIGNMENT).  status: optional device status word (see above).
  */
 int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_gscale,
                   const uint8_t* k_fp4, const uint8_t* k_sf, float k_gscale,
                   const float* w, int B, int T, int row0, int T_chunk,
                   int S, int k_bstride, int HI, int DI, int m,
                   const int32_t* q_pos0, void* score, int score_dtype, int score_ld,
-                  csa_stream_t stream);
+                  int32_t* status, csa_stream_t stream);
 
 /*
  * topk_select -- per query row, the k largest visible scores ([cf-1] §3.1
@@ -212,12 +221,14 @@ int topk_select_noalloc(const void* score, int score_dtype, int B, int T_chunk,
  *   sink fp32 [H] or NULL, lse fp32 [B, T, H] or NULL
  * Requires D in {64, 128}.  bf16 runs on tcgen05 and needs D = 128, H in
  * {64, 128} and k <= 1024 (else CSA_ERR_UNSUPPORTED); fp32 runs on CUDA cores.
+ * status: optional device status word (see above).
  */
 int sparse_attn_fwd(const void* q, const void* kv_c, const int32_t* idx,
                     const void* kv_raw, const float* sink, float tau, int W,
                     int B, int T, int row0, int T_chunk, int H, int D,
                     int kv_bstride, int k, int raw_cap, const int32_t* q_pos0,
-                    void* out, float* lse, int dtype, csa_stream_t stream);
+                    void* out, float* lse, int dtype, int32_t* status,
+                    csa_stream_t stream);
 
 /*
  * hca_dense_attn_fwd -- HCA attention ([cf-1] §3.2 dense attention over all
@@ -225,13 +236,14 @@ int sparse_attn_fwd(const void* q, const void* kv_c, const int32_t* idx,
  * with the entry set = every visible entry s < S (m*(s+1) - 1 <= p).
  *   kv_c [B, kv_bstride, D]
  * bf16 needs D = 128 and H in {16, 32, 64, 128}; fp32 runs on CUDA cores.
+ * status: optional device status word (see above).
  */
 int hca_dense_attn_fwd(const void* q, const void* kv_c, const void* kv_raw,
                        const float* sink, float tau, int W,
                        int B, int T, int row0, int T_chunk, int H, int D,
                        int kv_bstride, int S, int m, int raw_cap,
                        const int32_t* q_pos0, void* out, float* lse,
-                       int dtype, csa_stream_t stream);
+                       int dtype, int32_t* status, csa_stream_t stream);
 
 /*
  * swa_sink_merge -- the raw-window branch merged with a compressed-branch

@@ -8,7 +8,8 @@
 namespace csa {
 int launch_attn_tc(const void* q, const void* kv_c, const int32_t* idx, const void* kv_raw, const float* sink,
                    float tau, int W, int B, int Tq, int row0, int T_chunk, int H, int kv_bstride, int k, int S, int m,
-                   int raw_cap, const int32_t* q_pos0, void* out, float* lse, int sparse, cudaStream_t st);
+                   int raw_cap, const int32_t* q_pos0, void* out, float* lse, int sparse, int* status,
+                   cudaStream_t st);
 int launch_attn_simt(const void* q, const void* kv_c, const int32_t* idx, const void* kv_raw, const float* sink,
                      float tau, int W, int B, int Tq, int row0, int T_chunk, int H, int D, int kv_bstride, int k,
                      int S, int m, int raw_cap, const int32_t* q_pos0, void* out, float* lse, int dtype, int mode,
@@ -36,14 +37,14 @@ int check_attn_args(const void* q, const void* kv_c, const void* kv_raw, const i
 extern "C" int sparse_attn_fwd(const void* q, const void* kv_c, const int32_t* idx, const void* kv_raw,
                                const float* sink, float tau, int W, int B, int T, int row0, int T_chunk, int H,
                                int D, int kv_bstride, int k, int raw_cap, const int32_t* q_pos0, void* out,
-                               float* lse, int dtype, csa_stream_t stream) {
+                               float* lse, int dtype, int32_t* status, csa_stream_t stream) {
   int st = check_attn_args(q, kv_c, kv_raw, q_pos0, out, W, B, T, row0, T_chunk, H, D, raw_cap, dtype);
   if (st != CSA_OK) return st;
   CSA_REQUIRE(idx != nullptr && k >= 1 && kv_bstride >= 1, CSA_ERR_INVALID_ARG);
   if (dtype == CSA_BF16) {
     CSA_REQUIRE(D == 128, CSA_ERR_UNSUPPORTED);
     return launch_attn_tc(q, kv_c, idx, kv_raw, sink, tau, W, B, T, row0, T_chunk, H, kv_bstride, k, 0, 1, raw_cap,
-                          q_pos0, out, lse, 1, reinterpret_cast<cudaStream_t>(stream));
+                          q_pos0, out, lse, 1, status_word(status), reinterpret_cast<cudaStream_t>(stream));
   }
   return launch_attn_simt(q, kv_c, idx, kv_raw, sink, tau, W, B, T, row0, T_chunk, H, D, kv_bstride, k, 0, 1,
                           raw_cap, q_pos0, out, lse, dtype, 0, nullptr, nullptr,
@@ -53,14 +54,15 @@ extern "C" int sparse_attn_fwd(const void* q, const void* kv_c, const int32_t* i
 extern "C" int hca_dense_attn_fwd(const void* q, const void* kv_c, const void* kv_raw, const float* sink,
                                   float tau, int W, int B, int T, int row0, int T_chunk, int H, int D,
                                   int kv_bstride, int S, int m, int raw_cap, const int32_t* q_pos0, void* out,
-                                  float* lse, int dtype, csa_stream_t stream) {
+                                  float* lse, int dtype, int32_t* status, csa_stream_t stream) {
   int st = check_attn_args(q, kv_c, kv_raw, q_pos0, out, W, B, T, row0, T_chunk, H, D, raw_cap, dtype);
   if (st != CSA_OK) return st;
   CSA_REQUIRE(S >= 0 && kv_bstride >= S && m >= 1, CSA_ERR_INVALID_ARG);
   if (dtype == CSA_BF16) {
     CSA_REQUIRE(D == 128, CSA_ERR_UNSUPPORTED);
     return launch_attn_tc(q, kv_c, nullptr, kv_raw, sink, tau, W, B, T, row0, T_chunk, H, kv_bstride > 0 ? kv_bstride : 1,
-                          0, S, m, raw_cap, q_pos0, out, lse, 0, reinterpret_cast<cudaStream_t>(stream));
+                          0, S, m, raw_cap, q_pos0, out, lse, 0, status_word(status),
+                          reinterpret_cast<cudaStream_t>(stream));
   }
   return launch_attn_simt(q, kv_c, nullptr, kv_raw, sink, tau, W, B, T, row0, T_chunk, H, D, kv_bstride, 0, S,
                           m, raw_cap, q_pos0, out, lse, dtype, 1, nullptr, nullptr,

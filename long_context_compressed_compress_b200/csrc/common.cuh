@@ -21,9 +21,12 @@ int check_launch();                          // cudaGetLastError -> status
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Device-side error word: a bounded wait that gives up stores CSA_ERR_TIMEOUT
-// there (never traps); csa_device_status() reads and clears it.  Kernels get
-// its address as an argument; this returns it for the current device.
+// there (never traps).  A call may pass its own word; otherwise kernels get
+// the library's per-device word, which csa_device_status() reads and clears.
 int* device_status_ptr();
+inline int* status_word(int32_t* caller) { return caller != nullptr ? reinterpret_cast<int*>(caller) : device_status_ptr(); }
+// Wall-time limit of every bounded device wait (csa_set_wait_timeout_ns).
+uint64_t wait_limit_ns();
 
 // ------------------------------------------------------------- element access
 __device__ __forceinline__ float to_f(float x) { return x; }
@@ -152,17 +155,17 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait: gives up after kWaitNs of wall time (try_wait may suspend the
-// thread between polls, so the bound is on time, not on poll count), records
-// CSA_ERR_TIMEOUT | site << 8 in the status word and returns false; the caller
-// then skips its remaining work and tears down.
-constexpr uint64_t kWaitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int site = 0) {
+// Bounded wait: gives up after `limit_ns` of wall time (try_wait may suspend
+// the thread between polls, so the bound is on time, not on poll count),
+// records CSA_ERR_TIMEOUT | site << 8 in the status word and returns false;
+// the caller then skips its remaining work and tears down.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, uint64_t limit_ns,
+                                          int site = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitNs) break;
+    if (global_ns() - t0 > limit_ns) break;
   }
   atomicCAS(status, 0, CSA_ERR_TIMEOUT | (site << 8));
   return false;
@@ -198,15 +201,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, uint64_t tmap, int x, 
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
           "r"(dst),
       "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-// TMA 2D gather of four rows y0..y3 at column x (box one row high), no multicast.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, uint64_t tmap, int x, int y0, int y1, int y2, int y3,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(tmap), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
       : "memory");
 }
 // Make generic-proxy smem writes visible to the async proxy (tcgen05 reads).

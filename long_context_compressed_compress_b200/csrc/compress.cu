@@ -26,6 +26,9 @@ int* device_status_ptr() {
   return ptrs[dev];
 }
 
+static uint64_t g_wait_limit_ns = 0;   // 0: the default of 2 s
+uint64_t wait_limit_ns() { return g_wait_limit_ns ? g_wait_limit_ns : 2000000000ull; }
+
 int set_cuda_error(cudaError_t e) {
   t_last_cuda_error = static_cast<int>(e);
   return CSA_ERR_CUDA;
@@ -268,6 +271,11 @@ const char* csa_status_string(int status) {
 int csa_last_cuda_error(void) { return t_last_cuda_error; }
 
 int csa_version(void) { return 100; }
+
+int csa_set_wait_timeout_ns(uint64_t ns) {
+  g_wait_limit_ns = ns;
+  return CSA_OK;
+}
 
 int csa_device_status(int* status_out) {
   if (status_out == nullptr) return CSA_ERR_INVALID_ARG;

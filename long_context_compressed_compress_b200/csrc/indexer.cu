@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
     const uint8_t* __restrict__ q_fp4, const uint8_t* __restrict__ q_sf, const uint8_t* __restrict__ k_fp4,
     const uint8_t* __restrict__ k_sf, const float* __restrict__ w, float gscale, int T, int row0, int T_chunk,
     int S, int k_bstride, int DI, int m, const int32_t* __restrict__ q_pos0, TS* __restrict__ score, int ld,
-    int n_qtiles, int n_chunks, int* __restrict__ status) {
+    int n_qtiles, int n_chunks, int* __restrict__ status, unsigned long long wait_ns) {
   constexpr int TQ = NQ / HI;
   constexpr uint32_t kIdxTmemCols = IdxTmem<NQ>::cols;
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_kernel(
       if (sm.abort_flag) break;
       issue_mma(j);
     }
-    if (!mbar_wait(&sm.mbar[j % NB], static_cast<uint32_t>((j / NB) & 1), status)) sm.abort_flag = 1;
+    if (!mbar_wait(&sm.mbar[j % NB], static_cast<uint32_t>((j / NB) & 1), status, wait_ns)) sm.abort_flag = 1;
     tc_fence_after();
     // the MMA has consumed this stage: prefetch NS tiles ahead into it
     if (j + NS < ntiles) load_k_tile(et0 + j + NS, stage);
@@ -262,7 +262,8 @@ using namespace csa;
 extern "C" int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_gscale, const uint8_t* k_fp4,
                              const uint8_t* k_sf, float k_gscale, const float* w, int B, int T, int row0,
                              int T_chunk, int S, int k_bstride, int HI, int DI, int m, const int32_t* q_pos0,
-                             void* score, int score_dtype, int score_ld, csa_stream_t stream) {
+                             void* score, int score_dtype, int score_ld, int32_t* status_out,
+                             csa_stream_t stream) {
   CSA_REQUIRE(q_fp4 && q_sf && k_fp4 && k_sf && w && q_pos0 && score, CSA_ERR_INVALID_ARG);
   CSA_REQUIRE(B >= 0 && T >= 0 && row0 >= 0 && T_chunk >= 0 && row0 + T_chunk <= T, CSA_ERR_INVALID_ARG);
   CSA_REQUIRE(S >= 0 && k_bstride >= S && m >= 1 && score_ld >= S, CSA_ERR_INVALID_ARG);
@@ -288,8 +289,9 @@ extern "C" int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_
   const size_t floor_b = narrow ? IdxFloor<16>::bytes : IdxFloor<kWide>::bytes;
   const size_t smem = smem_min > floor_b ? smem_min : floor_b;
   const float g = q_gscale * k_gscale;
-  int* status = device_status_ptr();
+  int* status = status_word(status_out);
   CSA_REQUIRE(status != nullptr, CSA_ERR_CUDA);
+  const unsigned long long wait_ns = wait_limit_ns();
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 #define CSA_IDX_LAUNCH_NQ(HIV, TS, NQV)                                                                        \
   do {                                                                                                         \
@@ -297,7 +299,7 @@ extern "C" int indexer_score(const uint8_t* q_fp4, const uint8_t* q_sf, float q_
                          static_cast<int>(smem));                                                              \
     indexer_kernel<HIV, TS, NQV><<<static_cast<unsigned>(grid), kIdxThreads, smem, st>>>(                      \
         q_fp4, q_sf, k_fp4, k_sf, w, g, T, row0, T_chunk, S, k_bstride, DI, m, q_pos0, static_cast<TS*>(score), \
-        score_ld, n_qtiles, n_chunks, status);                                                                 \
+        score_ld, n_qtiles, n_chunks, status, wait_ns);                                                                 \
   } while (0)
 #define CSA_IDX_LAUNCH(HIV, TS)                                 \
   do {                                                          \

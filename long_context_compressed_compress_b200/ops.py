@@ -42,15 +42,16 @@ _SIGS = {
     "csa_last_cuda_error": ([], I),
     "csa_version": ([], I),
     "csa_device_status": ([ctypes.POINTER(I)], I),
+    "csa_set_wait_timeout_ns": ([ctypes.c_uint64], I),
     "csa_compress": ([P, P, P, I, I, I, I, I, I, P, I, P, I, P, P, F, P], I),
     "hca_compress": ([P, P, I, I, I, I, I, P, I, P], I),
     "nvfp4_quantize": ([P, I, I64, I, F, P, P, P], I),
-    "indexer_score": ([P, P, F, P, P, F, P, I, I, I, I, I, I, I, I, I, P, P, I, I, P], I),
+    "indexer_score": ([P, P, F, P, P, F, P, I, I, I, I, I, I, I, I, I, P, P, I, I, P, P], I),
     "topk_select": ([P, I, I, I, I, I, I, I, I, P, P, P, SZ, P], I),
     "topk_workspace_size": ([I, I, I, I], SZ),
     "topk_select_noalloc": ([P, I, I, I, I, I, I, I, I, P, P, P], I),
-    "sparse_attn_fwd": ([P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, P, P, P, I, P], I),
-    "hca_dense_attn_fwd": ([P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, I, P, P, P, I, P], I),
+    "sparse_attn_fwd": ([P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, P, P, P, I, P, P], I),
+    "hca_dense_attn_fwd": ([P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, I, P, P, P, I, P, P], I),
     "swa_sink_merge": ([P, P, P, P, P, F, I, I, I, I, I, I, I, I, P, P, I, P], I),
     "csa_ring_append": ([P, I, I, I, P, I, P, P], I),
     "csa_pos_advance": ([P, I, I, P], I),
@@ -93,9 +94,16 @@ def _check(fn, st):
 
 
 def device_status():
+    """Read and clear the library's per-device status word (calls given no
+    status word of their own report a timed-out wait there)."""
     v = I(0)
     _check("csa_device_status", lib.csa_device_status(ctypes.byref(v)))
     return v.value
+
+
+def set_wait_timeout_ns(ns):
+    """Wall-time limit of the kernels' bounded waits (0 = the default 2 s)."""
+    _check("csa_set_wait_timeout_ns", lib.csa_set_wait_timeout_ns(int(ns)))
 
 
 def csa_compress(a, b, z, m, out=None, out_fp4=None, out_sf=None, gscale=1.0, first_has_pred=0,
@@ -121,7 +129,7 @@ def nvfp4_quantize(x, packed, sf, gscale=1.0, stream=None):
 
 
 def indexer_score(q_fp4, q_sf, k_fp4, k_sf, w, q_pos0, score, S, m, row0=0, T_chunk=None, q_gscale=1.0,
-                  k_gscale=1.0, stream=None):
+                  k_gscale=1.0, status=None, stream=None):
     """q_fp4 [B,T,HI,DI/2], k_fp4 [B,k_bstride,DI/2], w [B,T,HI], score [B,T_chunk,ld]."""
     B, T, HI, half = q_fp4.shape
     DI = half * 2
@@ -129,7 +137,7 @@ def indexer_score(q_fp4, q_sf, k_fp4, k_sf, w, q_pos0, score, S, m, row0=0, T_ch
     _check("indexer_score", lib.indexer_score(
         _ptr(q_fp4), _ptr(q_sf), q_gscale, _ptr(k_fp4), _ptr(k_sf), k_gscale, _ptr(w), B, T, row0, T_chunk,
         S, k_fp4.shape[1], HI, DI, m, _ptr(q_pos0), _ptr(score), _dt(score), score.shape[-1],
-        _stream(stream)))
+        _ptr(status), _stream(stream)))
 
 
 def topk_select(score, idx, S, m, q_pos0, row0=0, workspace=None, stream=None):
@@ -154,24 +162,25 @@ def topk_workspace_size(B, T_chunk, S, k):
 
 
 def sparse_attn_fwd(q, kv_c, idx, kv_raw, sink, tau, W, q_pos0, out, lse=None, row0=0, T_chunk=None,
-                    raw_cap=None, stream=None):
+                    raw_cap=None, status=None, stream=None):
     B, T, H, D = q.shape
     T_chunk = T - row0 if T_chunk is None else T_chunk
     raw_cap = (kv_raw.shape[1] if kv_raw is not None else 1) if raw_cap is None else raw_cap
     _check("sparse_attn_fwd", lib.sparse_attn_fwd(
         _ptr(q), _ptr(kv_c), _ptr(idx), _ptr(kv_raw), _ptr(sink), tau, W, B, T, row0, T_chunk, H, D,
-        kv_c.shape[1], idx.shape[-1], raw_cap, _ptr(q_pos0), _ptr(out), _ptr(lse), _dt(q), _stream(stream)))
+        kv_c.shape[1], idx.shape[-1], raw_cap, _ptr(q_pos0), _ptr(out), _ptr(lse), _dt(q), _ptr(status),
+        _stream(stream)))
 
 
 def hca_dense_attn_fwd(q, kv_c, kv_raw, sink, tau, W, q_pos0, out, m, S=None, lse=None, row0=0, T_chunk=None,
-                       raw_cap=None, stream=None):
+                       raw_cap=None, status=None, stream=None):
     B, T, H, D = q.shape
     T_chunk = T - row0 if T_chunk is None else T_chunk
     S = kv_c.shape[1] if S is None else S
     raw_cap = (kv_raw.shape[1] if kv_raw is not None else 1) if raw_cap is None else raw_cap
     _check("hca_dense_attn_fwd", lib.hca_dense_attn_fwd(
         _ptr(q), _ptr(kv_c), _ptr(kv_raw), _ptr(sink), tau, W, B, T, row0, T_chunk, H, D, kv_c.shape[1], S, m,
-        raw_cap, _ptr(q_pos0), _ptr(out), _ptr(lse), _dt(q), _stream(stream)))
+        raw_cap, _ptr(q_pos0), _ptr(out), _ptr(lse), _dt(q), _ptr(status), _stream(stream)))
 
 
 def swa_sink_merge(o_c, lse_c, q, kv_raw, sink, tau, W, q_pos0, out, row0=0, T_chunk=None, raw_cap=None,

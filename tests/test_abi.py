@@ -65,16 +65,18 @@ def test_argument_validation_rejects_before_launch(lib):
     assert L.nvfp4_quantize(fake, 1, 4, 32, 0.0, fake, fake, None) == 1
     # indexer: unsupported DI / HI
     assert L.indexer_score(fake, fake, 1.0, fake, fake, 1.0, fake, 1, 64, 0, 64, 16, 16, 4, 48, 4, fake, fake,
-                           1, 16, None) == 2
+                           1, 16, None, None) == 2
     assert L.indexer_score(fake, fake, 1.0, fake, fake, 1.0, fake, 1, 64, 0, 64, 16, 16, 3, 64, 4, fake, fake,
-                           1, 16, None) == 2
+                           1, 16, None, None) == 2
     # attention: unsupported head dim
     assert L.sparse_attn_fwd(fake, fake, fake, fake, None, 1.0, 128, 1, 256, 0, 256, 8, 96, 64, 8, 256, fake,
-                             fake, None, 1, None) == 2
+                             fake, None, 1, None, None) == 2
     # window larger than the ring
     assert L.hca_dense_attn_fwd(fake, fake, fake, None, 1.0, 128, 1, 256, 0, 256, 8, 64, 2, 2, 128, 64, fake,
-                                fake, None, 1, None) == 1
+                                fake, None, 1, None, None) == 1
     # top-k: ld < S
     assert L.topk_select(fake, 1, 1, 4, 64, 32, 8, 4, 0, fake, fake, None, 0, None) == 1
     # empty problems are a no-op success
     assert L.topk_select(fake, 1, 0, 4, 64, 64, 8, 4, 0, fake, fake, None, 0, None) == 0
+    # the wait limit is a host setting (no device access)
+    assert L.csa_set_wait_timeout_ns(0) == 0

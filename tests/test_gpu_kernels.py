@@ -524,6 +524,38 @@ def test_attn_unsupported_shapes_rejected(ops):
         ops.sparse_attn_fwd(q, kv, idx, kv, None, 1.0, 0, pos0, torch.empty_like(q))
 
 
+def test_bounded_wait_timeout_reports_and_recovers(ops):
+    """With a 1 ns wait limit the attention kernel's first bounded wait gives
+    up: the kernel still returns, the call's own status word reads
+    CSA_ERR_TIMEOUT (the library's word stays clear), and with the limit
+    restored the same call on the same device gives the oracle's result."""
+    B, T, H, D, m, k, W = 1, 160, 64, 128, 4, 16, 128
+    S = T // m
+    tau = 1.0 / np.sqrt(D)
+    q, kv_c, raw, sink = _attn_inputs(B, T, H, D, S, "bf16", 95)
+    pos0 = torch.zeros((B,), dtype=torch.int32)
+    pos = np.arange(T)[None]
+    idx = oracle.topk_select(np.random.default_rng(6).standard_normal((B, T, S)), pos, m, k)
+    dq, dkv, draw, dsink, didx = q.cuda(), kv_c.cuda(), raw.cuda(), sink.cuda(), torch.from_numpy(idx).cuda()
+    out = torch.zeros_like(dq)
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    assert ops.device_status() == 0
+    ops.set_wait_timeout_ns(1)
+    try:
+        ops.sparse_attn_fwd(dq, dkv, didx, draw, dsink, tau, W, pos0.cuda(), out, status=status)
+        torch.cuda.synchronize()
+    finally:
+        ops.set_wait_timeout_ns(0)
+    assert int(status.item()) & 0xFF == 5, f"status {int(status.item()):#x}"
+    assert ops.device_status() == 0
+    status.zero_()
+    ops.sparse_attn_fwd(dq, dkv, didx, draw, dsink, tau, W, pos0.cuda(), out, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ro, _ = oracle.sparse_attn(q, kv_c, idx, raw, T, sink, tau, W, pos)
+    _attn_tol("bf16")(_np(out), oracle.round_out(ro, "bf16"))
+
+
 def test_no_device_timeouts(ops):
     torch.cuda.synchronize()
     assert ops.device_status() == 0
