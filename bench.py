@@ -477,6 +477,8 @@ def main():
             extra[name] = {k: sub[k] for k in ("value", "unit", "ms_per_step", "steps", "warmup", "config",
                                                "roofline", "kernels", "e2e", "gpu_launches", "clocks",
                                                "cpu_baseline") if k in sub}
+        extra["variants"] = measure_variants(args, rank, world, dev)
+        extra["kv_state"] = measure_state(args, rank, world, dev)
         line["workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -870,6 +872,114 @@ def measure_hca(args, rank, world, dev):
         line["cpu_baseline"] = hca_cpu_baseline(cfg, x)
     del x, lay
     return line
+
+
+def measure_variants(args, rank, world, dev):
+    """The same kernels at the variant settings the pages name: top-k 32 / 512
+    / 1024 on the CSA prefill workload and HCA ratio 64 on the HCA prefill
+    workload.  A short timed run each (inputs resident, per-kernel events);
+    tokens/s and the attention kernel's fraction of the bf16 burst peak."""
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import configs, inputs, layer
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    res = {}
+    cases = [("csa_prefill_32k_k32", configs.CSA_PREFILL_K32), ("csa_prefill_32k", configs.CSA_PREFILL),
+             ("csa_prefill_32k_k1024", configs.CSA_PREFILL_K1024),
+             ("hca_prefill_2x128k_ratio64", configs.HCA_PREFILL_M64)]
+    for name, cfg in cases:
+        x = inputs.layer_inputs(cfg, device="cuda")
+        lay = layer.CsaPrefill(cfg) if cfg.kind == "csa" else layer.HcaPrefill(cfg)
+        attn = "sparse_attn_fwd" if cfg.kind == "csa" else "hca_dense_attn_fwd"
+        ev = {}
+
+        @contextlib.contextmanager
+        def timer(nm):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            yield
+            e1.record(stream)
+            ev.setdefault(nm, []).append((e0, e1))
+
+        steps = 10 if cfg.kind == "csa" else 4
+        for _ in range(3):
+            lay.run(x)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(steps):
+            lay.run(x, timer=timer)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        ms = s0.elapsed_time(s1)
+        if world > 1:
+            ms = max_over_ranks(ms, dev)
+        kern = {k: sum(a.elapsed_time(b) for a, b in v) / steps for k, v in ev.items()}
+        fl = attn_flops(cfg)
+        tf = fl / (kern[attn] * 1e-3) / 1e12
+        res[name] = {"k" if cfg.kind == "csa" else "m": cfg.k if cfg.kind == "csa" else cfg.m,
+                     "value": job_throughput(world, cfg.B * cfg.T, ms / steps), "unit": "tokens/s",
+                     "ms_per_step": ms / steps, "steps": steps,
+                     "attention": {"kernel": attn, "ms": round(kern[attn], 4), "achieved": round(tf, 1),
+                                   "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4)},
+                     "kernels_ms": {k: round(v, 4) for k, v in kern.items()}}
+        del x, lay
+        torch.cuda.empty_cache()
+    return res
+
+
+def measure_state(args, rank, world, dev):
+    """KV-cache state management on the CSA prefill workload: the every-1024
+    snapshots of the raw window and compressor carries (one launch per tensor,
+    32 snapshots of B = 1, T = 32768) and one restore into a decode state.
+    Algorithmic bytes: each snapshot slot read once and written once."""
+    import dataclasses
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import configs, inputs, layer
+    cfg = configs.CSA_PREFILL
+    peaks = load_peaks()
+    x = inputs.layer_inputs(cfg, device="cuda")
+    pre = layer.CsaPrefill(cfg)
+    pre.run(x)
+    stream = torch.cuda.current_stream()
+    reps = 20
+    for _ in range(3):
+        ck = layer.PrefixCheckpoints(cfg, x)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        ck = layer.PrefixCheckpoints(cfg, x)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    if world > 1:
+        ms = max_over_ranks(ms, dev)
+    n = len(ck.positions)
+    bytes_ = 2 * 2 * cfg.B * n * (cfg.W * cfg.D + 2 * cfg.m * (3 * cfg.D + 3 * cfg.DI))
+    dcfg = dataclasses.replace(configs.CSA_DECODE, B=cfg.B, T0=ck.positions[-1] + 1, H=cfg.H, k=cfg.k, steps=4)
+    r0 = torch.cuda.Event(enable_timing=True)
+    r1 = torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    dec = ck.restore(dcfg, n - 1, pre.kv_c, pre.k_fp4, pre.k_sf, extra_entries=2)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    res = {"snapshots": n, "every": ck.every, "checkpoint_ms": round(ms, 5),
+           "checkpoint_bytes": bytes_, "checkpoint_GBps": round(bytes_ / (ms * 1e-3) / 1e9, 1),
+           "checkpoint_frac": round(bytes_ / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+           "restore_ms": round(r0.elapsed_time(r1), 4),
+           "restored_cache_entries": int(dec.cap), "launches": ck.launches}
+    del x, pre, ck, dec
+    return res
 
 
 def attn_flops(cfg):

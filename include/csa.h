@@ -270,6 +270,28 @@ int csa_ring_append(const void* rows, int dtype, int B, int D, void* ring,
                     int cap, const int32_t* pos, csa_stream_t stream);
 int csa_pos_advance(int32_t* pos, int B, int delta, csa_stream_t stream);
 
+/*
+ * csa_state_gather -- snapshots of a layer's decode-time state, the tier of
+ * the KV cache that is not the compressed entries themselves ([cf-1] §4.4:
+ * the sliding-window cache is checkpointed every 1024 tokens, so a request
+ * that shares a prefix restores that state instead of recomputing it).  For
+ * sequence b and snapshot c, with p = pos[b * npos + c] (the last token the
+ * snapshot covers):
+ *   window mode (m == 0): tokens j in (p - nrows, p]     (the raw window)
+ *   carry mode  (m >= 1): tokens j in [m (floor((p+1)/m) - 1), p]  (the last
+ *     complete block and the block in progress, which the next compressed
+ *     entries mix)
+ * are copied from src [B, src_cap, D] (token j at slot j % src_cap) into
+ * dst [B, npos, dst_cap, D] at slot j % dst_cap; every other slot of dst, and
+ * tokens j < 0, are written as zeros.  The same call restores a snapshot into
+ * a decode ring: src = the snapshot (src_cap = dst_cap), npos = 1.
+ * dtype CSA_F32 / CSA_BF16; D % 8 == 0; 16-byte aligned src and dst; dst_cap
+ * >= nrows (window) or >= 2m (carry).  Device memory owned by the caller.
+ */
+int csa_state_gather(const void* src, int dtype, int B, int D, int src_cap,
+                     const int32_t* pos, int npos, int m, int nrows,
+                     void* dst, int dst_cap, csa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

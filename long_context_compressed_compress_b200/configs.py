@@ -106,3 +106,17 @@ def scaled(cfg: LayerCfg, **kw) -> LayerCfg:
     d = dict(cfg.__dict__)
     d.update(kw)
     return LayerCfg(**d)
+
+
+# Variants of the same kernels named on the pages: HCA ratio 64
+# (devpress.csdn.net/awstech/6a462b3a… §3.1) and top-k 32 / 512 / 1024
+# (devpress.csdn.net/awstech/6a4623aa… attention paragraph; cf-1.com/news/5231315
+# §3.1; yfxerp.com/news/211352 §3 top_k_blocks).
+HCA_PREFILL_M64 = scaled(HCA_PREFILL, m=64)
+CSA_PREFILL_K32 = scaled(CSA_PREFILL, k=32)
+CSA_PREFILL_K1024 = scaled(CSA_PREFILL, k=1024)
+WORKLOADS.update({
+    "hca_prefill_2x128k_ratio64": HCA_PREFILL_M64,
+    "csa_prefill_32k_k32": CSA_PREFILL_K32,
+    "csa_prefill_32k_k1024": CSA_PREFILL_K1024,
+})

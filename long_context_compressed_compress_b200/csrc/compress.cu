@@ -244,6 +244,37 @@ __global__ void ring_append_kernel(const T* __restrict__ rows, int B, int D, T* 
     ring[(static_cast<size_t>(bi) * cap + slot) * D + c] = rows[static_cast<size_t>(bi) * D + c];
 }
 
+// One CTA per (sequence, snapshot); thread = (slot, 8-channel group).  Slot s
+// of the destination ring holds the token j <= p with j = s (mod dst_cap)
+// closest to p; it is copied when j lies in the snapshot's row range and is
+// >= 0, else zeroed, so every slot of the destination is written.
+template <typename T>
+__global__ void state_gather_kernel(const T* __restrict__ src, int D, int src_cap, const int32_t* __restrict__ pos,
+                                    int npos, int m, int nrows, T* __restrict__ dst, int dst_cap) {
+  const int snap = blockIdx.x;                 // b * npos + c
+  const int b = snap / npos;
+  const int p = pos[snap];
+  int lo;
+  if (m > 0) lo = m * ((p + 1) / m - 1);       // last complete block and the block in progress
+  else lo = p - nrows + 1;                     // the window
+  const int G = D >> 3;
+  for (int e = threadIdx.x; e < dst_cap * G; e += blockDim.x) {
+    const int sl = e / G, g = e - sl * G;
+    int d = (p - sl) % dst_cap;
+    if (d < 0) d += dst_cap;
+    const int j = p - d;
+    float v[8];
+    if (p >= 0 && j >= 0 && j >= lo) {
+      int ss = j % src_cap;
+      Vec8<T>::load(src + (static_cast<size_t>(b) * src_cap + ss) * D + 8 * g, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
+    Vec8<T>::store(dst + (static_cast<size_t>(snap) * dst_cap + sl) * D + 8 * g, v);
+  }
+}
+
 __global__ void pos_advance_kernel(int32_t* pos, int B, int delta) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < B) pos[i] += delta;
@@ -398,6 +429,28 @@ int csa_ring_append(const void* rows, int dtype, int B, int D, void* ring, int c
   else
     ring_append_kernel<__nv_bfloat16><<<B, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(rows), B, D,
                                                          static_cast<__nv_bfloat16*>(ring), cap, pos);
+  return check_launch();
+}
+
+int csa_state_gather(const void* src, int dtype, int B, int D, int src_cap, const int32_t* pos, int npos, int m,
+                     int nrows, void* dst, int dst_cap, csa_stream_t stream) {
+  CSA_REQUIRE(src && dst && pos, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(B >= 0 && npos >= 0 && D > 0 && src_cap > 0 && dst_cap > 0 && m >= 0, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(m > 0 ? dst_cap >= 2 * m : (nrows >= 1 && dst_cap >= nrows), CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(D % 8 == 0, CSA_ERR_UNSUPPORTED);
+  CSA_REQUIRE(aligned16(src) && aligned16(dst), CSA_ERR_ALIGNMENT);
+  const long long snaps = static_cast<long long>(B) * npos;
+  if (snaps == 0) return CSA_OK;
+  CSA_REQUIRE(snaps < (1ll << 31), CSA_ERR_UNSUPPORTED);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == CSA_F32)
+    state_gather_kernel<float><<<static_cast<unsigned>(snaps), 256, 0, st>>>(
+        static_cast<const float*>(src), D, src_cap, pos, npos, m, nrows, static_cast<float*>(dst), dst_cap);
+  else
+    state_gather_kernel<__nv_bfloat16><<<static_cast<unsigned>(snaps), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(src), D, src_cap, pos, npos, m, nrows, static_cast<__nv_bfloat16*>(dst),
+        dst_cap);
   return check_launch();
 }
 

@@ -149,13 +149,21 @@ class CsaDecode:
         self.kv_c = state["kv_c"]
         B, cap, D = self.kv_c.shape
         self.cap = cap
-        self.k_fp4 = torch.empty((B, cap, c.DI // 2), dtype=torch.uint8, device=device)
-        self.k_sf = torch.empty((B, cap, c.DI // 16), dtype=torch.uint8, device=device)
-        ops.nvfp4_quantize(state["k_I_src"], self.k_fp4, self.k_sf, gscale)
+        if "k_fp4" in state:
+            # keys already quantised (a cache restored from a prefill)
+            self.k_fp4, self.k_sf = state["k_fp4"], state["k_sf"]
+        else:
+            self.k_fp4 = torch.empty((B, cap, c.DI // 2), dtype=torch.uint8, device=device)
+            self.k_sf = torch.empty((B, cap, c.DI // 16), dtype=torch.uint8, device=device)
+            ops.nvfp4_quantize(state["k_I_src"], self.k_fp4, self.k_sf, gscale)
         self.ring = state["ring"]
         self.carry = {}
         slot0 = ((T0 // c.m - 1) % 2) * c.m      # the last complete block's slots
         for n in _CARRY:
+            if "carry_ring_" + n in state:
+                # a full 2m-slot carry ring (token j at slot j % 2m)
+                self.carry[n] = state["carry_ring_" + n]
+                continue
             src = state["carry_" + n]
             buf = torch.zeros((B, 2 * c.m, src.shape[-1]), dtype=dt, device=device)
             buf[:, slot0:slot0 + c.m] = src
@@ -231,6 +239,56 @@ class CsaDecode:
     def replay(self):
         self.graph.replay()
         return self.out
+
+
+class PrefixCheckpoints:
+    """Periodic snapshots of a CSA layer's decode-time state, taken from the
+    inputs of a prefill (cf-1.com/news/5231315 §4.4: the sliding-window cache
+    is checkpointed every 1024 tokens, so a request that shares a prefix
+    restores that state instead of recomputing it).
+
+    Snapshot c covers the tokens up to p_c = every * (c + 1) - 1 and holds the
+    raw window ring [B, n, W, D] and, for each compressor stream, the carry
+    ring [B, n, 2m, dim] (the last complete block and the block in progress),
+    in the decode layout (token j at slot j % cap).  The compressed entries and
+    NVFP4 keys of the prefix are not copied: once emitted they are final, so
+    the prefill's own buffers serve every snapshot (entries s < (p_c + 1) / m).
+    One ``csa_state_gather`` launch per tensor builds all snapshots."""
+
+    def __init__(self, cfg, x, every=1024, device="cuda"):
+        c = cfg
+        self.cfg, self.every = cfg, every
+        n = c.T // every
+        self.positions = [every * (i + 1) - 1 for i in range(n)]
+        self.pos = torch.tensor([self.positions] * c.B, dtype=torch.int32, device=device)
+        dt = x["kv_raw"].dtype
+        self.ring = torch.empty((c.B, n, c.W, c.D), dtype=dt, device=device)
+        ops.csa_state_gather(x["kv_raw"], self.pos, self.ring, m=0, nrows=c.W)
+        self.carry = {}
+        for name in _CARRY:
+            src = x[name]
+            buf = torch.empty((c.B, n, 2 * c.m, src.shape[-1]), dtype=dt, device=device)
+            ops.csa_state_gather(src, self.pos, buf, m=c.m)
+            self.carry[name] = buf
+        self.launches = 1 + len(_CARRY)
+
+    def restore(self, dcfg, i, kv_c, k_fp4, k_sf, extra_entries, device="cuda", with_lse=False):
+        """A CsaDecode positioned after snapshot i (next token p_i + 1), with a
+        cache of the prefix's entries plus room for ``extra_entries`` more."""
+        p = self.positions[i]
+        n_ent = (p + 1) // dcfg.m
+        B = kv_c.shape[0]
+        cap = n_ent + extra_entries
+        st = {"kv_c": torch.zeros((B, cap, kv_c.shape[-1]), dtype=kv_c.dtype, device=device),
+              "k_fp4": torch.zeros((B, cap, k_fp4.shape[-1]), dtype=torch.uint8, device=device),
+              "k_sf": torch.zeros((B, cap, k_sf.shape[-1]), dtype=torch.uint8, device=device),
+              "ring": self.ring[:, i].contiguous()}
+        st["kv_c"][:, :n_ent] = kv_c[:, :n_ent]
+        st["k_fp4"][:, :n_ent] = k_fp4[:, :n_ent]
+        st["k_sf"][:, :n_ent] = k_sf[:, :n_ent]
+        for name in _CARRY:
+            st["carry_ring_" + name] = self.carry[name][:, i].contiguous()
+        return CsaDecode(dcfg, st, p + 1, device=device, with_lse=with_lse)
 
 
 class Stack:

@@ -55,6 +55,7 @@ _SIGS = {
     "swa_sink_merge": ([P, P, P, P, P, F, I, I, I, I, I, I, I, I, P, P, I, P], I),
     "csa_ring_append": ([P, I, I, I, P, I, P, P], I),
     "csa_pos_advance": ([P, I, I, P], I),
+    "csa_state_gather": ([P, I, I, I, I, P, I, I, I, P, I, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -201,3 +202,16 @@ def csa_ring_append(rows, ring, pos, stream=None):
 
 def csa_pos_advance(pos, delta=1, stream=None):
     _check("csa_pos_advance", lib.csa_pos_advance(_ptr(pos), pos.numel(), delta, _stream(stream)))
+
+
+def csa_state_gather(src, pos, dst, m=0, nrows=0, src_cap=None, stream=None):
+    """Snapshot rows of a ring or a [B, T, D] stream into dst [B, npos, cap, D]
+    (see include/csa.h): window mode (m = 0, the last ``nrows`` tokens up to
+    pos) or carry mode (m >= 1, the last complete block and the one in
+    progress).  pos: int32 [B, npos] on the device."""
+    B, cap_src, D = src.shape
+    npos = pos.shape[-1]
+    dst_cap = dst.shape[-2]
+    _check("csa_state_gather", lib.csa_state_gather(
+        _ptr(src), _dt(src), B, D, cap_src if src_cap is None else src_cap, _ptr(pos), npos, m, nrows,
+        _ptr(dst), dst_cap, _stream(stream)))
