@@ -50,7 +50,7 @@ __all__ = [
     "csa_compress", "hca_compress", "nvfp4_quantize", "visible_entries",
     "indexer_score", "round_scores", "topk_select", "attend_rows",
     "sparse_attn", "dense_attn", "swa_sink_merge", "round_out",
-    "csa_layer", "hca_layer", "csa_decode_step",
+    "csa_layer", "hca_layer", "csa_decode_step", "grouped_out_proj",
 ]
 
 
@@ -453,3 +453,28 @@ def csa_decode_step(st, x, p, m, k, W, tau, dtype, gscale=1.0):
     out, lse = sparse_attn(q, st["kv_c"], idx, st["ring"], W, x["sink"], tau, W, pos)
     return {"out": round_out(out, dtype)[:, 0], "lse": formats.f32(lse)[:, 0], "idx": idx[:, 0],
             "score": sc[:, 0]}
+
+
+# ---------------------------------------------------------------------------
+# (6) grouped output projection ([cf-1] §3.4: with many query heads -- 128 --
+# the heads are split into groups, each group's concatenated head outputs are
+# projected to a smaller dimension, and the concatenation of the groups is
+# projected to the model dimension, which cuts the projection's parameters and
+# FLOPs against one projection of all H*D values).
+# ---------------------------------------------------------------------------
+def grouped_out_proj(o, w1, w2, dtype="bf16"):
+    """o [..., H, D] attention output; w1 [g, d_g, (H/g)*D] (group j's
+    projection, rows = output features); w2 [d_model, g*d_g].
+        y[..., j*d_g:(j+1)*d_g] = o[..., heads of group j, :].flatten() @ w1[j].T
+        out = y @ w2.T
+    y is rounded once to ``dtype`` (it is stored between the two products), and
+    so is the result.  Returns (y, out) as float64 arrays of the rounded values."""
+    o, w1, w2 = _f64(o), _f64(w1), _f64(w2)
+    g, d_g, kg = w1.shape
+    H, D = o.shape[-2], o.shape[-1]
+    assert H % g == 0 and kg == (H // g) * D
+    lead = o.shape[:-2]
+    x = o.reshape(*lead, g, kg)                                    # group j = heads [j H/g, (j+1) H/g)
+    y = np.concatenate([x[..., j, :] @ w1[j].T for j in range(g)], axis=-1)
+    y = round_out(y, dtype)
+    return y, round_out(y @ w2.T, dtype)

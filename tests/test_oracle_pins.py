@@ -458,3 +458,52 @@ def test_decode_entry0_differs_from_a_zero_predecessor():
     slab = [np.concatenate([np.zeros((1, m, cfg.D)), x[n][:, :m].double().numpy()], axis=1) for n in ("a", "b", "z")]
     wrong = oracle.round_out(oracle.csa_compress(slab[0], slab[1], slab[2], m, first_has_pred=True), "f32")
     assert np.abs(wrong[:, 0] - st["kv_c"][:, 0]).max() > 1e-3
+
+
+# ------------------------------------------------------- grouped out projection
+
+def test_grouped_out_proj_one_group_is_the_plain_two_stage_projection():
+    """g = 1: y = o.flatten() @ w1[0].T, out = y @ w2.T (torch matmul, fp64)."""
+    o = RNG.standard_normal((5, 4, 8))
+    w1 = RNG.standard_normal((1, 6, 32))
+    w2 = RNG.standard_normal((7, 6))
+    y, out = oracle.grouped_out_proj(o, w1, w2, dtype="f32")
+    yt = torch.from_numpy(o.reshape(5, 32)) @ torch.from_numpy(w1[0]).T
+    np.testing.assert_allclose(y, formats.f32(yt.numpy()), rtol=1e-6)
+    np.testing.assert_allclose(out, formats.f32((torch.from_numpy(y) @ torch.from_numpy(w2).T).numpy()),
+                               rtol=1e-6)
+
+
+def test_grouped_out_proj_identity_groups_reduce_to_one_projection():
+    """Each w1 block the identity (d_g = (H/g) D): the result is the ungrouped
+    output projection o.flatten() @ w2.T, i.e. the grouping only regroups."""
+    T, H, D, g = 6, 8, 4, 4
+    o = RNG.standard_normal((T, H, D))
+    kg = H // g * D
+    w1 = np.stack([np.eye(kg) for _ in range(g)])
+    w2 = RNG.standard_normal((5, g * kg))
+    _, out = oracle.grouped_out_proj(o, w1, w2, dtype="f32")
+    ref = (torch.from_numpy(o.reshape(T, H * D)) @ torch.from_numpy(w2).T).numpy()
+    # y is stored (rounded to fp32) between the products: the gap is within
+    # fp32 rounding of the 32-term sums
+    np.testing.assert_allclose(out, formats.f32(ref), rtol=1e-5, atol=1e-5)
+
+
+def test_grouped_out_proj_groups_follow_head_order():
+    """Group j is heads [j H/g, (j+1) H/g): zeroing group 1's heads in o zeroes
+    exactly group 1's slice of y; permuting the groups (heads, w1 blocks and
+    w2 column blocks together) leaves the result unchanged."""
+    T, H, D, g, dg = 3, 8, 2, 4, 3
+    o = RNG.standard_normal((T, H, D))
+    w1 = RNG.standard_normal((g, dg, H // g * D))
+    w2 = RNG.standard_normal((4, g * dg))
+    o0 = o.copy()
+    o0[:, 2:4] = 0.0
+    y0, _ = oracle.grouped_out_proj(o0, w1, w2, dtype="f32")
+    assert np.all(y0[:, dg:2 * dg] == 0) and np.all(y0[:, :dg] != 0)
+    perm = [2, 0, 3, 1]
+    op = np.concatenate([o[:, 2 * j:2 * j + 2] for j in perm], axis=1)
+    w2p = np.concatenate([w2[:, dg * j:dg * j + dg] for j in perm], axis=1)
+    _, out = oracle.grouped_out_proj(o, w1, w2, dtype="f32")
+    _, outp = oracle.grouped_out_proj(op, w1[perm], w2p, dtype="f32")
+    np.testing.assert_allclose(outp, out, rtol=1e-6, atol=1e-9)
