@@ -479,6 +479,7 @@ def main():
                                                "cpu_baseline") if k in sub}
         extra["variants"] = measure_variants(args, rank, world, dev)
         extra["kv_state"] = measure_state(args, rank, world, dev)
+        extra["grouped_out_proj"] = measure_outproj(args, rank, world, dev)
         line["workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -979,6 +980,52 @@ def measure_state(args, rank, world, dev):
            "restore_ms": round(r0.elapsed_time(r1), 4),
            "restored_cache_entries": int(dec.cap), "launches": ck.launches}
     del x, pre, ck, dec
+    return res
+
+
+def measure_outproj(args, rank, world, dev):
+    """Grouped output projection after a 128-head attention layer: M = 32768
+    rows, H = 128 x D = 128, 8 groups of 16 heads projected to 1024 each, then
+    to a model dimension of 4096 (two tcgen05 GEMM launches; bf16 in, fp32
+    accumulation).  Algorithmic FLOPs: 2 M (H D d_g + g d_g d_model)."""
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import ops
+    peaks = load_peaks()
+    M, H, D, g, d_g, d_model = 32768, 128, 128, 8, 1024, 4096
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(9)
+    o = torch.randn((M, H, D), generator=gen, device="cuda").to(torch.bfloat16)
+    w1 = (torch.randn((g, d_g, H // g * D), generator=gen, device="cuda") / (H // g * D) ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn((d_model, g * d_g), generator=gen, device="cuda") / (g * d_g) ** 0.5).to(torch.bfloat16)
+    y = torch.empty((M, g * d_g), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((M, d_model), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        ops.grouped_out_proj(o, w1, w2, y, out)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    reps = 10
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        ops.grouped_out_proj(o, w1, w2, y, out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    if world > 1:
+        ms = max_over_ranks(ms, dev)
+    flops = 2.0 * M * (H * D * d_g + g * d_g * d_model)
+    plain = 2.0 * M * H * D * d_model
+    tf = flops / (ms * 1e-3) / 1e12
+    res = {"M": M, "H": H, "D": D, "groups": g, "d_g": d_g, "d_model": d_model, "ms": round(ms, 4),
+           "achieved": round(tf, 1), "unit": "TFLOP/s", "peak": peaks["bf16_tflops"],
+           "frac": round(tf / peaks["bf16_tflops"], 4), "flops": flops,
+           "flops_vs_ungrouped": round(flops / plain, 3), "launches": 2}
+    del o, w1, w2, y, out
+    torch.cuda.empty_cache()
     return res
 
 

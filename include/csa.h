@@ -261,6 +261,26 @@ int swa_sink_merge(const void* o_c, const float* lse_c, const void* q,
                    csa_stream_t stream);
 
 /*
+ * grouped_out_proj -- the grouped output projection after the attention
+ * ([cf-1] §3.4: with many query heads -- 128 -- the heads are split into
+ * groups, each group's concatenated head outputs are projected to a smaller
+ * dimension, and the concatenation of the groups is projected to the model
+ * dimension, cutting the projection's parameters and FLOPs):
+ *   y[:, j d_g : (j+1) d_g] = o[:, heads [j H/g, (j+1) H/g), :] . w1[j]^T
+ *   out = y . w2^T
+ *   o [M, H, D] bf16 (the attention output, M = B * T rows)
+ *   w1 [groups, d_g, (H/groups) D] bf16, w2 [d_model, groups d_g] bf16
+ *   y [M, groups d_g] bf16 (caller-owned intermediate), out [M, d_model] bf16
+ * Two launches of one tcgen05 GEMM (fp32 accumulation in TMEM, bf16 stores);
+ * y is rounded to bf16 between the products.  Requires (H/groups) D % 64 == 0,
+ * d_g % 256 == 0 and d_model % 256 == 0 (else CSA_ERR_UNSUPPORTED), 16-byte
+ * aligned tensors.  status: optional device status word (see above).
+ */
+int grouped_out_proj(const void* o, int M, int H, int D, int groups, int d_g,
+                     const void* w1, const void* w2, int d_model, void* y,
+                     void* out, int32_t* status, csa_stream_t stream);
+
+/*
  * Decode-step helpers (state update of the KV cache tiers, [cf-1] §4.4):
  * csa_ring_append writes rows[b, :] (dtype, [B, D]) into ring[b, pos[b] % cap, :];
  * csa_pos_advance adds delta to each pos[b].  Both read positions on the device,

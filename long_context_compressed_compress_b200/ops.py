@@ -56,6 +56,7 @@ _SIGS = {
     "csa_ring_append": ([P, I, I, I, P, I, P, P], I),
     "csa_pos_advance": ([P, I, I, P], I),
     "csa_state_gather": ([P, I, I, I, I, P, I, I, I, P, I, P], I),
+    "grouped_out_proj": ([P, I, I, I, I, I, P, P, I, P, P, P, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -215,3 +216,14 @@ def csa_state_gather(src, pos, dst, m=0, nrows=0, src_cap=None, stream=None):
     _check("csa_state_gather", lib.csa_state_gather(
         _ptr(src), _dt(src), B, D, cap_src if src_cap is None else src_cap, _ptr(pos), npos, m, nrows,
         _ptr(dst), dst_cap, _stream(stream)))
+
+
+def grouped_out_proj(o, w1, w2, y, out, status=None, stream=None):
+    """o [..., H, D] bf16 -> y [M, g*d_g], out [M, d_model] (see include/csa.h);
+    w1 [g, d_g, (H/g)*D], w2 [d_model, g*d_g]."""
+    H, D = o.shape[-2], o.shape[-1]
+    M = o.numel() // (H * D)
+    g, d_g, _ = w1.shape
+    _check("grouped_out_proj", lib.grouped_out_proj(
+        _ptr(o), M, H, D, g, d_g, _ptr(w1), _ptr(w2), w2.shape[0], _ptr(y), _ptr(out), _ptr(status),
+        _stream(stream)))
