@@ -59,7 +59,8 @@ def parse():
     ap.add_argument("--T", type=int, default=0,
                     help="profiling case: override the layer's token count (not a bench line)")
     ap.add_argument("--workload", default="csa_prefill_32k",
-                    choices=["csa_prefill_32k", "csa_decode_32x1m", "hca_prefill_2x128k", "stack_hhcc_256k"],
+                    choices=["csa_prefill_32k", "csa_decode_32x1m", "hca_prefill_2x128k", "stack_hhcc_256k",
+                             "grouped_out_proj_32k"],
                     help="csa_prefill_32k (the default line), csa_decode_32x1m (decode steps/s), "
                          "hca_prefill_2x128k (HCA prefill tokens/s) or stack_hhcc_256k (4-layer prefill stack)")
     ap.add_argument("--no-extra", action="store_true",
@@ -305,6 +306,9 @@ def main():
         return
     if args.workload == "stack_hhcc_256k":
         main_stack(args, rank, world, local)
+        return
+    if args.workload == "grouped_out_proj_32k":
+        main_outproj(args, rank, world, local)
         return
     if args.impl == "reference":
         run_reference(args, cfg, rank)
@@ -983,6 +987,36 @@ def measure_state(args, rank, world, dev):
     return res
 
 
+def main_outproj(args, rank, world, local):
+    """The grouped output projection as a line of its own (see ``measure_outproj``)."""
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import build
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps({"impl": "reference", "unavailable": "no CPU timing of a 3.3 TFLOP projection; "
+                              "its oracle runs on sampled rows in the tests"}), flush=True)
+        return
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    r = measure_outproj(args, rank, world, dev)
+    line = {"metric": METRIC, "value": r["achieved"], "unit": "TFLOP/s", "n_gpus": world, "steps": r["reps"],
+            "warmup": 3, "ms_per_step": r["ms"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) activations, scaled N(0,1) weights)",
+            "config": {"workload": "grouped_out_proj_32k", **{k: r[k] for k in ("M", "H", "D", "groups", "d_g",
+                                                                                 "d_model")}},
+            "roofline": {"bound": "tensor", "kernel": "gemm_kernel", "achieved": r["achieved"], "peak": r["peak"],
+                         "unit": "TFLOP/s", "frac": r["frac"], "traffic": None},
+            "gpu_launches": r["launches"] * r["reps"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def measure_outproj(args, rank, world, dev):
     """Grouped output projection after a 128-head attention layer: M = 32768
     rows, H = 128 x D = 128, 8 groups of 16 heads projected to 1024 each, then
@@ -1006,7 +1040,7 @@ def measure_outproj(args, rank, world, dev):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    reps = 10
+    reps = max(2, min(args.steps, 10))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -1023,7 +1057,7 @@ def measure_outproj(args, rank, world, dev):
     res = {"M": M, "H": H, "D": D, "groups": g, "d_g": d_g, "d_model": d_model, "ms": round(ms, 4),
            "achieved": round(tf, 1), "unit": "TFLOP/s", "peak": peaks["bf16_tflops"],
            "frac": round(tf / peaks["bf16_tflops"], 4), "flops": flops,
-           "flops_vs_ungrouped": round(flops / plain, 3), "launches": 2}
+           "flops_vs_ungrouped": round(flops / plain, 3), "launches": 2, "reps": reps}
     del o, w1, w2, y, out
     torch.cuda.empty_cache()
     return res

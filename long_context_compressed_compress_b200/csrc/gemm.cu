@@ -77,7 +77,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   const Args& a = args;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sm.abort_flag;
-  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+  // N tiles vary fastest: the CTAs sharing an A row block (every N tile of a
+  // group, or of the whole row) run together and read it once from DRAM
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
   const int a_k0 = a.group_k > 0 ? (n0 / a.group_n) * a.group_k : 0;
   const int nk = (a.group_k > 0 ? a.group_k : a.K) / BK;
 
@@ -233,7 +235,8 @@ int gm_launch(const void* A, int lda, int K_a, const void* B, int ldb, int K_b, 
     if (e != cudaSuccess) return set_cuda_error(e);
     attr_set = true;
   }
-  dim3 grid((M + BM - 1) / BM, N / BN);
+  CSA_REQUIRE((M + BM - 1) / BM < 65536, CSA_ERR_UNSUPPORTED);
+  dim3 grid(N / BN, (M + BM - 1) / BM);
   gemm_kernel<<<grid, kThreads, smem, st>>>(a, maps);
   return check_launch();
 }
