@@ -96,6 +96,8 @@ def algorithmic_work(cfg):
         "indexer_flops": B * 2.0 * vis_pairs * HI * DI,
         "indexer_bytes": B * (vis_pairs * esz + T * HI * (DI // 2 + DI // 16 + 4) + S * (DI // 2 + DI // 16)),
         "topk_bytes": B * (vis_pairs * esz + T * k * 4),
+        # fused indexer -> top-k: its inputs once and the indices; no score bytes
+        "indexer_topk_bytes": B * (T * HI * (DI // 2 + DI // 16 + 4) + S * (DI // 2 + DI // 16) + T * k * 4),
         "compress_bytes": B * (3 * T * D * esz + S * D * esz),
         "compress_keys_bytes": B * (3 * T * DI * esz + S * (DI // 2 + DI // 16)),
         "quant_bytes": B * (T * HI * DI * esz + T * HI * (DI // 2 + DI // 16)),
@@ -430,6 +432,7 @@ def main():
         "nvfp4_quantize": ("GB/s", work["quant_bytes"]),
         "indexer_score": ("GB/s", work["indexer_bytes"]),
         "topk_select": ("GB/s", work["topk_bytes"]),
+        "indexer_topk": ("GB/s", work["indexer_topk_bytes"]),
         "sparse_attn_fwd": ("TFLOP/s", work["attn_flops"]),
     }
     kernels = {}
@@ -484,6 +487,7 @@ def main():
         extra["variants"] = measure_variants(args, rank, world, dev)
         extra["kv_state"] = measure_state(args, rank, world, dev)
         extra["grouped_out_proj"] = measure_outproj(args, rank, world, dev)
+        extra["indexer_topk"] = measure_fused_topk(args, rank, world, dev)
         line["workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -1059,6 +1063,53 @@ def measure_outproj(args, rank, world, dev):
            "frac": round(tf / peaks["bf16_tflops"], 4), "flops": flops,
            "flops_vs_ungrouped": round(flops / plain, 3), "launches": 2, "reps": reps}
     del o, w1, w2, y, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_fused_topk(args, rank, world, dev):
+    """Indexer score + top-k on the CSA prefill shapes (T = 32768, S = 8192,
+    k = 512): the fused kernel (scores kept on chip) against indexer_score +
+    topk_select (BF16 scores through HBM), on the same NVFP4 inputs, with the
+    two index tensors compared bit for bit."""
+    import torch
+    import torch.distributed as dist
+    from long_context_compressed_compress_b200 import configs, inputs, layer, ops
+    cfg = configs.CSA_PREFILL
+    lay = layer.CsaPrefill(cfg, fused=False)
+    x = inputs.layer_inputs(cfg, device="cuda")
+    lay.run(x)
+    torch.cuda.synchronize()
+    idx_f = torch.empty_like(lay.idx)
+    stream = torch.cuda.current_stream()
+
+    def fused():
+        ops.indexer_topk(lay.q_fp4, lay.q_sf, lay.k_fp4, lay.k_sf, x["w"], lay.q_pos0, idx_f, cfg.S, cfg.m)
+
+    def unfused():
+        ops.indexer_score(lay.q_fp4, lay.q_sf, lay.k_fp4, lay.k_sf, x["w"], lay.q_pos0, lay.score, cfg.S, cfg.m)
+        ops.topk_select(lay.score, lay.idx, cfg.S, cfg.m, lay.q_pos0)
+
+    res = {"config": "csa_prefill_32k (T 32768, S 8192, k 512, HI 4)"}
+    reps = max(2, min(args.steps, 10))
+    for name, fn in (("fused_ms", fused), ("unfused_ms", unfused)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        res[name] = round(max_over_ranks(ms, dev) if world > 1 else ms, 4)
+    res["bit_identical"] = bool(torch.equal(idx_f, lay.idx))
+    res["launches"] = {"fused": 1, "unfused": 2}
+    del lay, x, idx_f
     torch.cuda.empty_cache()
     return res
 

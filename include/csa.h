@@ -183,6 +183,30 @@ int topk_select(const void* score, int score_dtype, int B, int T_chunk, int S,
 size_t topk_workspace_size(int B, int T_chunk, int S, int k);
 
 /*
+ * indexer_topk -- indexer score and top-k selection in one kernel ([cf-1]
+ * §3.1 the lightning indexer scores every visible compressed entry and each
+ * query keeps its top-k; §4.4 the index score is BF16).  The result equals
+ * topk_select applied to the BF16 scores indexer_score writes for the same
+ * inputs, bit for bit (same arithmetic, rounding, keys, tie rule and output
+ * order); the score matrix is never written.
+ *   q_fp4, q_sf, w, k_fp4, k_sf, q_pos0, row0, T_chunk, S, m: as indexer_score
+ *   idx int32 [B, T_chunk, k]: as topk_select
+ * Requires DI = 64, HI in {4, 8} and S <= indexer_topk_max_entries(HI, DI)
+ * (the visible scores of 8 query rows are held on chip), else
+ * CSA_ERR_UNSUPPORTED: callers then use indexer_score + topk_select.  Same
+ * alignment rules as indexer_score.  status: optional device status word
+ * (see above).
+ */
+int indexer_topk(const uint8_t* q_fp4, const uint8_t* q_sf, float q_gscale,
+                 const uint8_t* k_fp4, const uint8_t* k_sf, float k_gscale,
+                 const float* w, int B, int T, int row0, int T_chunk,
+                 int S, int k_bstride, int HI, int DI, int m,
+                 const int32_t* q_pos0, int32_t* idx, int k,
+                 int32_t* status, csa_stream_t stream);
+/* Largest S indexer_topk accepts on the current device (0: HI/DI unsupported). */
+int indexer_topk_max_entries(int HI, int DI);
+
+/*
  * topk_select_noalloc -- topk_select for callers that cannot allocate device
  * memory (no workspace argument).  The pages have no counterpart to this call;
  * it exists only for allocator-free callers.  Same arguments, layouts, result

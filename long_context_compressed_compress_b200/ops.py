@@ -48,6 +48,8 @@ _SIGS = {
     "nvfp4_quantize": ([P, I, I64, I, F, P, P, P], I),
     "indexer_score": ([P, P, F, P, P, F, P, I, I, I, I, I, I, I, I, I, P, P, I, I, P, P], I),
     "topk_select": ([P, I, I, I, I, I, I, I, I, P, P, P, SZ, P], I),
+    "indexer_topk": ([P, P, F, P, P, F, P, I, I, I, I, I, I, I, I, I, P, P, I, P, P], I),
+    "indexer_topk_max_entries": ([I, I], I),
     "topk_workspace_size": ([I, I, I, I], SZ),
     "topk_select_noalloc": ([P, I, I, I, I, I, I, I, I, P, P, P], I),
     "sparse_attn_fwd": ([P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, P, P, P, I, P, P], I),
@@ -148,6 +150,22 @@ def topk_select(score, idx, S, m, q_pos0, row0=0, workspace=None, stream=None):
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("topk_select", lib.topk_select(_ptr(score), _dt(score), B, T_chunk, S, ld, k, m, row0,
                                           _ptr(q_pos0), _ptr(idx), _ptr(workspace), ws, _stream(stream)))
+
+
+def indexer_topk(q_fp4, q_sf, k_fp4, k_sf, w, q_pos0, idx, S, m, row0=0, T_chunk=None, q_gscale=1.0,
+                 k_gscale=1.0, status=None, stream=None):
+    """Indexer score and top-k in one kernel: idx [B,T_chunk,k] equals
+    topk_select of the BF16 scores indexer_score would write."""
+    B, T, HI, half = q_fp4.shape
+    DI = half * 2
+    T_chunk = T - row0 if T_chunk is None else T_chunk
+    _check("indexer_topk", lib.indexer_topk(
+        _ptr(q_fp4), _ptr(q_sf), q_gscale, _ptr(k_fp4), _ptr(k_sf), k_gscale, _ptr(w), B, T, row0, T_chunk,
+        S, k_fp4.shape[1], HI, DI, m, _ptr(q_pos0), _ptr(idx), idx.shape[-1], _ptr(status), _stream(stream)))
+
+
+def indexer_topk_max_entries(HI, DI):
+    return int(lib.indexer_topk_max_entries(HI, DI))
 
 
 def topk_select_noalloc(score, idx, S, m, q_pos0, row0=0, stream=None):

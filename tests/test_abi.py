@@ -68,6 +68,16 @@ def test_argument_validation_rejects_before_launch(lib):
                            1, 16, None, None) == 2
     assert L.indexer_score(fake, fake, 1.0, fake, fake, 1.0, fake, 1, 64, 0, 64, 16, 16, 3, 64, 4, fake, fake,
                            1, 16, None, None) == 2
+    # fused indexer + top-k: DI other than 64, HI outside {4, 8}, null idx, k < 1
+    assert L.indexer_topk(fake, fake, 1.0, fake, fake, 1.0, fake, 1, 64, 0, 64, 16, 16, 4, 32, 4, fake, fake, 8,
+                          None, None) == 2
+    assert L.indexer_topk(fake, fake, 1.0, fake, fake, 1.0, fake, 1, 64, 0, 64, 16, 16, 2, 64, 4, fake, fake, 8,
+                          None, None) == 2
+    assert L.indexer_topk(fake, fake, 1.0, fake, fake, 1.0, fake, 1, 64, 0, 64, 16, 16, 4, 64, 4, fake, None, 8,
+                          None, None) == 1
+    assert L.indexer_topk(fake, fake, 1.0, fake, fake, 1.0, fake, 1, 64, 0, 64, 16, 16, 4, 64, 4, fake, fake, 0,
+                          None, None) == 1
+    assert L.indexer_topk_max_entries(4, 32) == 0
     # attention: unsupported head dim
     assert L.sparse_attn_fwd(fake, fake, fake, fake, None, 1.0, 128, 1, 256, 0, 256, 8, 96, 64, 8, 256, fake,
                              fake, None, 1, None, None) == 2

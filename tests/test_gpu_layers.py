@@ -54,11 +54,11 @@ def _out_check(got, ref, dtype):
         assert err <= 2e-2, f"bf16 max-abs {err:.3e}"
 
 
-def check_csa(L, cfg, rows=None, chunk=None):
+def check_csa(L, cfg, rows=None, chunk=None, fused=None):
     dev = "cuda"
     x = inputs.layer_inputs(cfg, device="cpu")
     xd = {k: v.to(dev) for k, v in x.items()}
-    lay = L.CsaPrefill(cfg, chunk=chunk)
+    lay = L.CsaPrefill(cfg, chunk=chunk, fused=fused)
     idx_all = torch.empty((cfg.B, cfg.T, cfg.k), dtype=torch.int32, device=dev)
     out = lay.run(xd, keep_idx=idx_all)
     torch.cuda.synchronize()
@@ -101,13 +101,16 @@ def test_pr1_fp32_layer_full(L):
     assert ov >= 0.995
 
 
-def test_csa_bf16_small_layer(L):
+@pytest.mark.parametrize("fused", [True, False])
+def test_csa_bf16_small_layer(L, fused):
+    """Scores and selection fused in one kernel, or written and read back."""
     cfg = configs.scaled(configs.CSA_PREFILL, T=4096, seed=11)
-    check_csa(L, cfg, rows=sample_rows(1, cfg.T, 256, 512), chunk=1536)
+    check_csa(L, cfg, rows=sample_rows(1, cfg.T, 256, 512), chunk=1536, fused=fused)
 
 
-def test_csa_bf16_full_size_sampled(L):
-    check_csa(L, configs.CSA_PREFILL, rows=sample_rows(1, configs.CSA_PREFILL.T), chunk=8192)
+@pytest.mark.parametrize("fused", [False, True])
+def test_csa_bf16_full_size_sampled(L, fused):
+    check_csa(L, configs.CSA_PREFILL, rows=sample_rows(1, configs.CSA_PREFILL.T), chunk=8192, fused=fused)
 
 
 def check_hca(L, cfg, rows):
