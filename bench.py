@@ -67,6 +67,8 @@ def parse():
                          "hca_prefill_2x128k (HCA prefill tokens/s) or stack_hhcc_256k (4-layer prefill stack)")
     ap.add_argument("--no-extra", action="store_true",
                     help="default run only: skip the decode and HCA measurements under 'workloads'")
+    ap.add_argument("--fused", action="store_true",
+                    help="CSA prefill: score and select in the fused indexer_topk kernel")
     return ap.parse_args()
 
 
@@ -336,7 +338,7 @@ def main():
     peaks = load_peaks()
     work = algorithmic_work(cfg)
     x = inputs.layer_inputs(cfg, device="cuda")
-    lay = layer.CsaPrefill(cfg, chunk=args.chunk or None)
+    lay = layer.CsaPrefill(cfg, chunk=args.chunk or None, fused=args.fused)
     stream = torch.cuda.current_stream()
 
     # per-kernel CUDA events on the launching stream, inside the timed region
@@ -389,7 +391,7 @@ def main():
     d2h = outs_host[0].numel() * outs_host[0].element_size()
     e2e_ms = float("nan")
     if args.e2e_steps > 0:
-        lays = [lay, layer.CsaPrefill(cfg, chunk=args.chunk or None)]
+        lays = [lay, layer.CsaPrefill(cfg, chunk=args.chunk or None, fused=args.fused)]
         xds = [{k: torch.empty_like(v) for k, v in x.items()} for _ in range(2)]
         e2e_ms = pipelined_e2e(lays, host, xds, outs_host, args.e2e_steps, world)
         barrier()
@@ -446,7 +448,8 @@ def main():
         "data": "synthetic (seeded N(0,1) inputs, U(0,1) indexer weights, N(0,1) sink)",
         "config": {"workload": "csa_prefill_32k", "B": cfg.B, "T": cfg.T, "H": cfg.H, "D": cfg.D, "m": cfg.m,
                    "S": cfg.S, "k": cfg.k, "HI": cfg.HI, "DI": cfg.DI, "W": cfg.W,
-                   "chunk": lay.chunk, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "chunk": lay.chunk, "indexer_topk": "fused" if lay.fused else "two kernels",
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (q + out = 1.07 GB per step)"},
         # no end-to-end number when no e2e step was timed (--e2e-steps 0)
         "e2e": {"value": job_throughput(world, tokens, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
