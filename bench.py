@@ -468,7 +468,7 @@ def main():
     if not args.no_extra and not args.T:
         # the metric's other two throughputs, measured in the same run (every
         # rank runs them, in the same order, as independent replicas)
-        del x, xd, host, lay
+        del x, host, outs_host, lay
         torch.cuda.empty_cache()
         extra = {}
         for name, fn in (("csa_decode_32x1m", measure_decode), ("hca_prefill_2x128k", measure_hca)):
