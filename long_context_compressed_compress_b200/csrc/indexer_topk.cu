@@ -526,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_topk_kernel(const __grid_
       for (int u = 0; u < 2; ++u) nv[u] = 2 * tp + u < gr.ntok ? visible(gr.pbase, 2 * tp + u, a) : 0;
       uint16_t* krow0 = keys + static_cast<size_t>(2 * tp) * a.npad;
       uint32_t rm[2] = {0u, 0u};
-      uint32_t v[2][2][CPW];   // [pipeline slot][tile][column]
+      uint32_t v[2][2][CPW];   // [chunk of the pair][tile][column]
       auto load = [&](int cg, uint32_t (&dst)[2][CPW]) {
         const uint32_t col = tmem + lane_base + (cg % NACC) * 2 * N + tp * CPW;
 #pragma unroll
@@ -560,53 +560,34 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_topk_kernel(const __grid_
           kr[128] = static_cast<uint16_t>(k2 >> 16);
         }
       };
-      // software pipeline: the TMEM loads of chunk c + 1 overlap the keys of chunk c
+      // two chunks per synchronisation: the later chunk's commit covers both
+      // (the MMA thread commits in order), one TMEM load wait for four tiles
       const int nch = gr.nch;
-      if (nch > 0) {
-        ok = waitw(&sm.acc_full[gc % NACC], (gc / NACC) & 1, a, abort_flag, 6);
-        if (ok) {
-          tc_fence_after();
-          load(gc, v[0]);
-          tmem_ld_wait();
-          reg_fence(v[0][0]);
-          reg_fence(v[0][1]);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.acc_empty[gc % NACC]);
-        }
-      }
 #pragma unroll 1
       for (int c = 0; ok && c < nch; c += 2) {
-        // chunk c (global gc + c) is in v[0]
-        const int g1 = gc + c + 1;
-        if (c + 1 < nch) {
-          if (!waitw(&sm.acc_full[g1 % NACC], (g1 / NACC) & 1, a, abort_flag, 6)) { ok = false; break; }
-          tc_fence_after();
-          load(g1, v[1]);
+        const int g0 = gc + c;
+        const bool two = c + 1 < nch;
+        const int gl = two ? g0 + 1 : g0;
+        if (!waitw(&sm.acc_full[gl % NACC], (gl / NACC) & 1, a, abort_flag, 6)) {
+          ok = false;
+          break;
         }
-        consume(c, v[0]);
-        if (c + 1 >= nch) break;
+        tc_fence_after();
+        load(g0, v[0]);
+        if (two) load(g0 + 1, v[1]);
         tmem_ld_wait();
+        reg_fence(v[0][0]);
+        reg_fence(v[0][1]);
         reg_fence(v[1][0]);
         reg_fence(v[1][1]);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.acc_empty[g1 % NACC]);
-        // chunk c + 1 is in v[1]
-        const int g2 = g1 + 1;
-        if (c + 2 < nch) {
-          if (!waitw(&sm.acc_full[g2 % NACC], (g2 / NACC) & 1, a, abort_flag, 6)) { ok = false; break; }
-          tc_fence_after();
-          load(g2, v[0]);
+        if (lane == 0) {
+          mbar_arrive(&sm.acc_empty[g0 % NACC]);
+          if (two) mbar_arrive(&sm.acc_empty[(g0 + 1) % NACC]);
         }
-        consume(c + 1, v[1]);
-        if (c + 2 >= nch) break;
-        tmem_ld_wait();
-        reg_fence(v[0][0]);
-        reg_fence(v[0][1]);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.acc_empty[g2 % NACC]);
+        consume(c, v[0]);
+        if (two) consume(c + 1, v[1]);
       }
       gc += nch;
       // each row's largest key: this warp's 32 lanes x 2 tiles
