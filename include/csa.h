@@ -138,6 +138,34 @@ int nvfp4_quantize(const void* x, int in_dtype, int64_t rows, int D, float gscal
                    uint8_t* packed, uint8_t* sf, csa_stream_t stream);
 
 /*
+ * csa_decode_update -- one decode step's cache update in one launch (the
+ * per-step work of [cf-1] §3.1 compression and §3.3 window for token p =
+ * pos[b] of every sequence b), with the results of this call sequence:
+ *   csa_ring_append of a, b, z, a_I, b_I, z_I into their 2m-slot carry rings,
+ *   csa_compress (decode mode) of the KV entry into kv_c,
+ *   csa_compress (decode mode, NVFP4 out) of the indexer key into k_fp4/k_sf,
+ *   csa_ring_append of kv_raw into the W-slot window ring,
+ *   nvfp4_quantize of q_I into q_fp4/q_sf (global scale gscale, also used
+ *   for the keys).
+ *   a, b, z, kv_raw [B, D]; a_I, b_I, z_I [B, DI]; q_I [B, HI, DI]   (this step)
+ *   carry_* [B, 2m, D or DI], ring [B, W, D], kv_c [B, cap, D],
+ *   k_fp4 [B, cap, DI/2], k_sf [B, cap, DI/16], q_fp4 [B, HI, DI/2], q_sf [B, HI, DI/16]
+ * An entry whose index is >= cap is dropped.  Requires dtype CSA_BF16,
+ * D and DI multiples of 16, DI <= 256 and (D/8 + 31)/32 + 1 + (HI DI/8 + 31)/32
+ * <= 8 (else CSA_ERR_UNSUPPORTED; the separate calls serve other shapes);
+ * 16-byte aligned rows, rings, q_I and kv_c.  pos is not advanced.
+ */
+int csa_decode_update(const void* a, const void* b, const void* z,
+                      const void* a_I, const void* b_I, const void* z_I,
+                      const void* kv_raw, const void* q_I, int dtype, int B,
+                      int D, int DI, int HI, int m, int W, int cap,
+                      void* carry_a, void* carry_b, void* carry_z,
+                      void* carry_aI, void* carry_bI, void* carry_zI, void* ring,
+                      void* kv_c, uint8_t* k_fp4, uint8_t* k_sf,
+                      uint8_t* q_fp4, uint8_t* q_sf, float gscale,
+                      const int32_t* pos, csa_stream_t stream);
+
+/*
  * indexer_score -- lightning-indexer score over compressed entries ([cf-1]
  * §3.1 lightning indexer, §3.4 FP4 QK; [yfxerp] indexer_rank 64):
  *   score[b,r,s] = sum_h w[b,row0+r,h] * ReLU( qhat[b,row0+r,h,:] . khat[b,s,:] )

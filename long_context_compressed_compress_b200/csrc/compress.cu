@@ -1,7 +1,8 @@
 // Streaming kernels of the CSA/HCA layer: the gated overlapping 4:1 compressor
 // (cf-1.com/news/5231315 §3.1), the 128:1 compressor (§3.2), NVFP4 block
 // quantisation of the indexer QK path (§3.4, §4.4), and the decode-state
-// helpers (ring append, position advance; §4.4 KV cache tiers).
+// helpers (ring append, position advance, the fused per-step state update;
+// §4.4 KV cache tiers).
 //
 // All of these are HBM-bound: one thread owns 8 channels of one entry and
 // moves 16-byte vectors, consecutive threads cover consecutive channels so a
@@ -36,6 +37,63 @@ int set_cuda_error(cudaError_t e) {
 int check_launch() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? CSA_OK : set_cuda_error(e);
+}
+
+// ---------------------------------------------------------------------------
+// The gated pooling of one compressed entry for 8 channels (one thread): the
+// per-channel max of the 2m gate logits, then the exp-weighted sums of a over
+// the block's rows cur0 .. cur0 + m - 1 and of b over the predecessor's rows
+// pred0 .. (when has_pred), in fp32; the result rounded to Tout.  a, b, z
+// point at the thread's 8 channels of row 0 of its slab.  Shared by the
+// compressor and the fused decode-state update, so both give the same bits.
+// ---------------------------------------------------------------------------
+template <typename Tin, typename Tout>
+__device__ __forceinline__ void pool_entry8(const Tin* __restrict__ a, const Tin* __restrict__ b,
+                                            const Tin* __restrict__ zb, int D, int m, int cur0, int pred0,
+                                            int has_pred, bool active, float e8[8]) {
+  float mx[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
+  float v[8];
+  if (active) {
+    for (int r = 0; r < m; ++r) {
+      Vec8<Tin>::load(zb + static_cast<size_t>(cur0 + r) * D, v);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], v[c]);
+      if (has_pred) {
+        Vec8<Tin>::load(zb + static_cast<size_t>(pred0 + r) * D, v);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], v[c]);
+      }
+    }
+  }
+  float sum[8], acc[8], x[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) { sum[c] = 0.f; acc[c] = 0.f; }
+  if (active) {
+    for (int r = 0; r < m; ++r) {
+      Vec8<Tin>::load(zb + static_cast<size_t>(cur0 + r) * D, v);
+      Vec8<Tin>::load(a + static_cast<size_t>(cur0 + r) * D, x);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float e = expf(v[c] - mx[c]);
+        sum[c] += e;
+        acc[c] = fmaf(e, x[c], acc[c]);
+      }
+      if (has_pred) {
+        Vec8<Tin>::load(zb + static_cast<size_t>(pred0 + r) * D, v);
+        Vec8<Tin>::load(b + static_cast<size_t>(pred0 + r) * D, x);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float e = expf(v[c] - mx[c]);
+          sum[c] += e;
+          acc[c] = fmaf(e, x[c], acc[c]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) e8[c] = active ? round_to(__fdiv_rn(acc[c], sum[c]), (Tout*)nullptr) : 0.f;
 }
 
 // ---------------------------------------------------------------------------
@@ -82,51 +140,8 @@ __global__ void __launch_bounds__(256) csa_compress_kernel(
   }
   const int rows = decode ? 2 * m : T;
   const size_t slab = static_cast<size_t>(bi) * rows * D + static_cast<size_t>(cg) * 8;
-  const Tin* zb = z + slab;
-  float mx[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
-  float v[8];
-  if (active) {
-    for (int r = 0; r < m; ++r) {
-      Vec8<Tin>::load(zb + static_cast<size_t>(cur0 + r) * D, v);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], v[c]);
-      if (has_pred) {
-        Vec8<Tin>::load(zb + static_cast<size_t>(pred0 + r) * D, v);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mx[c] = fmaxf(mx[c], v[c]);
-      }
-    }
-  }
-  float sum[8], acc[8], x[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) { sum[c] = 0.f; acc[c] = 0.f; }
-  if (active) {
-    for (int r = 0; r < m; ++r) {
-      Vec8<Tin>::load(zb + static_cast<size_t>(cur0 + r) * D, v);
-      Vec8<Tin>::load(a + slab + static_cast<size_t>(cur0 + r) * D, x);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float e = expf(v[c] - mx[c]);
-        sum[c] += e;
-        acc[c] = fmaf(e, x[c], acc[c]);
-      }
-      if (has_pred) {
-        Vec8<Tin>::load(zb + static_cast<size_t>(pred0 + r) * D, v);
-        Vec8<Tin>::load(b + slab + static_cast<size_t>(pred0 + r) * D, x);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float e = expf(v[c] - mx[c]);
-          sum[c] += e;
-          acc[c] = fmaf(e, x[c], acc[c]);
-        }
-      }
-    }
-  }
   float e8[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) e8[c] = active ? round_to(__fdiv_rn(acc[c], sum[c]), (Tout*)nullptr) : 0.f;
+  pool_entry8<Tin, Tout>(a + slab, b + slab, z + slab, D, m, cur0, pred0, has_pred, active, e8);
   const size_t orow = static_cast<size_t>(bi) * out_bstride + static_cast<size_t>(eidx);
   if (out != nullptr && active) Vec8<Tout>::store(out + orow * D + cg * 8, e8);
   if (out_fp4 != nullptr) {
@@ -280,6 +295,113 @@ __global__ void pos_advance_kernel(int32_t* pos, int B, int delta) {
   if (i < B) pos[i] += delta;
 }
 
+
+// ---------------------------------------------------------------------------
+// Fused decode-state update, one CTA per sequence: the work of six compressor
+// carry appends, the raw-window append, the two decode-mode compressions and
+// the q_I quantisation of one decode step, in one launch with the same results
+// (the same pooling and NVFP4 code as the separate kernels).
+//   threads [0, 3 G + 3 GI + G) : 16-byte copies of this step's rows into the
+//                                 carry rings (slot p % 2m) and the window ring
+//                                 (slot p % W)
+//   warps   [0, wk)             : the KV entry, one thread per 8 channels
+//   warp    wk                  : the indexer key entry + NVFP4 (GI <= 32)
+//   warps   [wq, wq + nq)       : q_I -> NVFP4, one thread per 8 values
+// ---------------------------------------------------------------------------
+struct DecodeUpdateArgs {
+  const void* row[7];        // a, b, z, a_I, b_I, z_I, kv_raw: [B, D or DI]
+  void* ring[7];             // carry rings [B, 2m, D or DI] (x6), window ring [B, W, D]
+  const void* q_I;           // [B, HI, DI]
+  void* kv_c;                // [B, cap, D]
+  uint8_t* k_fp4;            // [B, cap, DI/2]
+  uint8_t* k_sf;             // [B, cap, DI/16]
+  uint8_t* q_fp4;            // [B, HI, DI/2]
+  uint8_t* q_sf;             // [B, HI, DI/16]
+  const int32_t* pos;
+  int D, DI, HI, m, W, cap, wk, wq;
+  float g;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) decode_update_kernel(const DecodeUpdateArgs args) {
+  const DecodeUpdateArgs& a = args;
+  const int bi = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int p = a.pos[bi];
+  const int G = a.D >> 3, GI = a.DI >> 3;
+  // ---- appends (16 bytes = 8 elements per thread and copy)
+  const int cslot = p % (2 * a.m), rslot = p % a.W;
+  for (int v = tid; v < 3 * G + 3 * GI + G; v += blockDim.x) {
+    int s, off, width, slot, cap;
+    if (v < 3 * G) {
+      s = v / G; off = v - s * G; width = a.D; slot = cslot; cap = 2 * a.m;
+    } else if (v < 3 * G + 3 * GI) {
+      const int u = v - 3 * G;
+      s = 3 + u / GI; off = u - (u / GI) * GI; width = a.DI; slot = cslot; cap = 2 * a.m;
+    } else {
+      s = 6; off = v - 3 * G - 3 * GI; width = a.D; slot = rslot; cap = a.W;
+    }
+    const uint4 x = reinterpret_cast<const uint4*>(static_cast<const T*>(a.row[s]) + static_cast<size_t>(bi) * width)[off];
+    reinterpret_cast<uint4*>(static_cast<T*>(a.ring[s]) + (static_cast<size_t>(bi) * cap + slot) * width)[off] = x;
+  }
+  __syncthreads();
+  // ---- the entry (p + 1) / m - 1 when this token completes its block
+  const int i = (p + 1) / a.m - 1;
+  const bool emit = ((p + 1) % a.m == 0) && i >= 0 && i < a.cap;
+  const int cur0 = (i & 1) * a.m, pred0 = ((i + 1) & 1) * a.m;
+  const int has_pred = i > 0;
+  if (warp < a.wk) {
+    const int cg = tid;
+    if (cg < G) {
+      const size_t slab = static_cast<size_t>(bi) * 2 * a.m * a.D + static_cast<size_t>(cg) * 8;
+      float e8[8];
+      pool_entry8<T, T>(static_cast<const T*>(a.ring[0]) + slab, static_cast<const T*>(a.ring[1]) + slab,
+                        static_cast<const T*>(a.ring[2]) + slab, a.D, a.m, cur0, pred0, has_pred, emit, e8);
+      if (emit) Vec8<T>::store(static_cast<T*>(a.kv_c) + (static_cast<size_t>(bi) * a.cap + i) * a.D + cg * 8, e8);
+    }
+  } else if (warp == a.wk) {
+    const int cg = lane;
+    const bool act = emit && cg < GI;
+    const size_t slab = static_cast<size_t>(bi) * 2 * a.m * a.DI + static_cast<size_t>(cg < GI ? cg : 0) * 8;
+    float e8[8];
+    pool_entry8<T, T>(static_cast<const T*>(a.ring[3]) + slab, static_cast<const T*>(a.ring[4]) + slab,
+                      static_cast<const T*>(a.ring[5]) + slab, a.DI, a.m, cur0, pred0, has_pred, act, e8);
+    // 16-element NVFP4 block = this lane's 8 channels + its neighbour's
+    float am = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) am = fmaxf(am, fabsf(e8[c]));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    uint32_t sfb;
+    const uint32_t codes = nvfp4_encode8(e8, am, a.g, &sfb);
+    if (act) {
+      const size_t orow = static_cast<size_t>(bi) * a.cap + i;
+      reinterpret_cast<uint32_t*>(a.k_fp4 + orow * (a.DI / 2))[cg] = codes;
+      if ((cg & 1) == 0) a.k_sf[orow * (a.DI / 16) + (cg >> 1)] = static_cast<uint8_t>(sfb);
+    }
+  } else if (warp >= a.wq) {
+    // ---- q_I of this sequence: HI * DI / 8 threads of 8 values
+    const int n8 = a.HI * a.DI / 8;
+    const int u = tid - 32 * a.wq;
+    const bool ok = u < n8;
+    const long long gid = static_cast<long long>(bi) * n8 + (ok ? u : 0);
+    float v[8];
+    if (ok) {
+      Vec8<T>::load(static_cast<const T*>(a.q_I) + gid * 8, v);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v[c] = 0.f;
+    }
+    float am = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) am = fmaxf(am, fabsf(v[c]));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    uint32_t sfb;
+    const uint32_t codes = nvfp4_encode8(v, am, a.g, &sfb);
+    if (ok) {
+      reinterpret_cast<uint32_t*>(a.q_fp4)[gid] = codes;
+      if ((gid & 1) == 0) a.q_sf[gid >> 1] = static_cast<uint8_t>(sfb);
+    }
+  }
+}
 }  // namespace csa
 
 using namespace csa;
@@ -413,6 +535,57 @@ int nvfp4_quantize(const void* x, int in_dtype, int64_t rows, int D, float gscal
   else
     nvfp4_quantize_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), bs, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), n8, gscale, packed, sf);
+  return check_launch();
+}
+
+int csa_decode_update(const void* a, const void* b, const void* z, const void* a_I, const void* b_I,
+                      const void* z_I, const void* kv_raw, const void* q_I, int dtype, int B, int D, int DI, int HI,
+                      int m, int W, int cap, void* carry_a, void* carry_b, void* carry_z, void* carry_aI,
+                      void* carry_bI, void* carry_zI, void* ring, void* kv_c, uint8_t* k_fp4, uint8_t* k_sf,
+                      uint8_t* q_fp4, uint8_t* q_sf, float gscale, const int32_t* pos, csa_stream_t stream) {
+  CSA_REQUIRE(a && b && z && a_I && b_I && z_I && kv_raw && q_I && pos, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(carry_a && carry_b && carry_z && carry_aI && carry_bI && carry_zI && ring, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(kv_c && k_fp4 && k_sf && q_fp4 && q_sf, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(B >= 0 && m >= 1 && m <= 16 && W >= 1 && cap >= 1 && HI >= 1 && gscale > 0.f, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(dtype == CSA_F32 || dtype == CSA_BF16, CSA_ERR_INVALID_ARG);
+  CSA_REQUIRE(D > 0 && DI > 0 && D % 16 == 0 && DI % 16 == 0, CSA_ERR_UNSUPPORTED);
+  const int esz = dtype == CSA_F32 ? 4 : 2;
+  const int G = D / 8, GI = DI / 8;
+  // 8 elements per 16-byte copy: bf16 rows only (fp32 rows take the separate calls)
+  CSA_REQUIRE(esz == 2, CSA_ERR_UNSUPPORTED);
+  const int wk = (G + 31) / 32;
+  const int wq = wk + 1;
+  const int n8 = HI * DI / 8;
+  CSA_REQUIRE(GI <= 32 && wq + (n8 + 31) / 32 <= 8, CSA_ERR_UNSUPPORTED);
+  const void* rows[7] = {a, b, z, a_I, b_I, z_I, kv_raw};
+  void* rings[7] = {carry_a, carry_b, carry_z, carry_aI, carry_bI, carry_zI, ring};
+  for (int i = 0; i < 7; ++i) CSA_REQUIRE(aligned16(rows[i]) && aligned16(rings[i]), CSA_ERR_ALIGNMENT);
+  CSA_REQUIRE(aligned16(q_I) && aligned16(kv_c) && (reinterpret_cast<uintptr_t>(k_fp4) & 3u) == 0 &&
+                  (reinterpret_cast<uintptr_t>(q_fp4) & 3u) == 0,
+              CSA_ERR_ALIGNMENT);
+  if (B == 0) return CSA_OK;
+  DecodeUpdateArgs args{};
+  for (int i = 0; i < 7; ++i) {
+    args.row[i] = rows[i];
+    args.ring[i] = rings[i];
+  }
+  args.q_I = q_I;
+  args.kv_c = kv_c;
+  args.k_fp4 = k_fp4;
+  args.k_sf = k_sf;
+  args.q_fp4 = q_fp4;
+  args.q_sf = q_sf;
+  args.pos = pos;
+  args.D = D;
+  args.DI = DI;
+  args.HI = HI;
+  args.m = m;
+  args.W = W;
+  args.cap = cap;
+  args.wk = wk;
+  args.wq = wq;
+  args.g = gscale;
+  decode_update_kernel<__nv_bfloat16><<<B, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(args);
   return check_launch();
 }
 

@@ -144,6 +144,7 @@ class CsaDecode:
         csa_compress (decode, NVFP4)  the same entry's indexer key        -> k_I
         csa_ring_append               token p's raw KV -> ring slot p % W
         nvfp4_quantize                q_I
+          (these five lines are one csa_decode_update launch for bf16 caches)
         indexer_score                 score [B, 1, cap] (visible prefix only)
         topk_select                   idx [B, 1, k] (multi-CTA rows, workspace)
         sparse_attn_fwd               out [B, 1, H, D] (window + sink fused)
@@ -153,7 +154,7 @@ class CsaDecode:
     captured once in a CUDA graph (``capture``) and replayed.
     """
 
-    def __init__(self, cfg, state, T0, device="cuda", gscale=1.0, with_lse=False):
+    def __init__(self, cfg, state, T0, device="cuda", gscale=1.0, with_lse=False, fused_update=None):
         self.cfg = c = cfg
         dt = _DT[c.dtype]
         self.dt = dt
@@ -193,8 +194,12 @@ class CsaDecode:
         nws = ops.topk_workspace_size(B, 1, cap, c.k)
         self.ws = torch.empty((max(1, nws // 4),), dtype=torch.int32, device=device) if nws else None
         self.sink = state.get("sink")
+        # the cache update of a step (7 appends, 2 compressions, the q_I
+        # quantisation) in one launch where the shapes allow (bf16)
+        can_fuse = c.dtype == "bf16" and c.D % 16 == 0 and c.DI % 16 == 0 and c.DI <= 256
+        self.fused_update = can_fuse if fused_update is None else bool(fused_update)
         # multi-CTA top-k: workspace memset + three kernels
-        self.launches = 6 + 2 + 1 + 1 + 1 + (4 if nws else 1) + 1 + 1
+        self.launches = (1 if self.fused_update else 6 + 2 + 1 + 1) + 1 + (4 if nws else 1) + 1 + 1
         self.graph = None
         self.x = None
 
@@ -203,20 +208,25 @@ class CsaDecode:
         ``sink`` [H] if the state has none).  Returns out [B, 1, H, D]."""
         c = self.cfg
         t = timer or _no_timer
-        for n in _CARRY:
+        if self.fused_update:
+            with t("csa_decode_update"):
+                ops.csa_decode_update(x, self.carry, self.ring, self.kv_c, self.k_fp4, self.k_sf, self.q_fp4,
+                                      self.q_sf, self.pos, c.m, self.g)
+        else:
+            for n in _CARRY:
+                with t("csa_ring_append"):
+                    ops.csa_ring_append(x[n], self.carry[n], self.pos)
+            with t("csa_compress"):
+                ops.csa_compress(self.carry["a"], self.carry["b"], self.carry["z"], c.m, out=self.kv_c,
+                                 ring_pos=self.pos, out_bstride=self.cap)
+            with t("csa_compress_indexer_keys"):
+                ops.csa_compress(self.carry["a_I"], self.carry["b_I"], self.carry["z_I"], c.m,
+                                 out_fp4=self.k_fp4, out_sf=self.k_sf, gscale=self.g, ring_pos=self.pos,
+                                 out_bstride=self.cap, out_dtype=self.dt)
             with t("csa_ring_append"):
-                ops.csa_ring_append(x[n], self.carry[n], self.pos)
-        with t("csa_compress"):
-            ops.csa_compress(self.carry["a"], self.carry["b"], self.carry["z"], c.m, out=self.kv_c,
-                             ring_pos=self.pos, out_bstride=self.cap)
-        with t("csa_compress_indexer_keys"):
-            ops.csa_compress(self.carry["a_I"], self.carry["b_I"], self.carry["z_I"], c.m, out_fp4=self.k_fp4,
-                             out_sf=self.k_sf, gscale=self.g, ring_pos=self.pos, out_bstride=self.cap,
-                             out_dtype=self.dt)
-        with t("csa_ring_append"):
-            ops.csa_ring_append(x["kv_raw"], self.ring, self.pos)
-        with t("nvfp4_quantize"):
-            ops.nvfp4_quantize(x["q_I"], self.q_fp4, self.q_sf, self.g)
+                ops.csa_ring_append(x["kv_raw"], self.ring, self.pos)
+            with t("nvfp4_quantize"):
+                ops.nvfp4_quantize(x["q_I"], self.q_fp4, self.q_sf, self.g)
         with t("indexer_score"):
             ops.indexer_score(self.q_fp4, self.q_sf, self.k_fp4, self.k_sf, x["w"].view(-1, 1, c.HI), self.pos,
                               self.score, self.cap, c.m, q_gscale=self.g, k_gscale=self.g)

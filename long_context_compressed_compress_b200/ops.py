@@ -57,6 +57,7 @@ _SIGS = {
     "swa_sink_merge": ([P, P, P, P, P, F, I, I, I, I, I, I, I, I, P, P, I, P], I),
     "csa_ring_append": ([P, I, I, I, P, I, P, P], I),
     "csa_pos_advance": ([P, I, I, P], I),
+    "csa_decode_update": ([P] * 8 + [I] * 8 + [P] * 12 + [F, P, P], I),
     "csa_state_gather": ([P, I, I, I, I, P, I, I, I, P, I, P], I),
     "grouped_out_proj": ([P, I, I, I, I, I, P, P, I, P, P, P, P], I),
 }
@@ -217,6 +218,20 @@ def csa_ring_append(rows, ring, pos, stream=None):
     B, D = rows.shape
     _check("csa_ring_append", lib.csa_ring_append(_ptr(rows), _dt(rows), B, D, _ptr(ring), ring.shape[1],
                                                   _ptr(pos), _stream(stream)))
+
+
+def csa_decode_update(x, carry, ring, kv_c, k_fp4, k_sf, q_fp4, q_sf, pos, m, gscale=1.0, stream=None):
+    """One decode step's cache update in one launch (see the C header):
+    ``x`` holds this step's rows a, b, z, a_I, b_I, z_I, kv_raw [B, .] and
+    q_I [B, HI, DI]; ``carry`` the six 2m-slot carry rings by name."""
+    B, D = x["a"].shape[0], x["a"].shape[-1]
+    DI = x["a_I"].shape[-1]
+    HI = x["q_I"].shape[-2]
+    names = ("a", "b", "z", "a_I", "b_I", "z_I")
+    _check("csa_decode_update", lib.csa_decode_update(
+        *[_ptr(x[n]) for n in names], _ptr(x["kv_raw"]), _ptr(x["q_I"]), _dt(x["a"]), B, D, DI, HI, m,
+        ring.shape[1], kv_c.shape[1], *[_ptr(carry[n]) for n in names], _ptr(ring), _ptr(kv_c), _ptr(k_fp4),
+        _ptr(k_sf), _ptr(q_fp4), _ptr(q_sf), gscale, _ptr(pos), _stream(stream)))
 
 
 def csa_pos_advance(pos, delta=1, stream=None):

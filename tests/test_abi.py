@@ -78,6 +78,8 @@ def test_argument_validation_rejects_before_launch(lib):
     assert L.indexer_topk(fake, fake, 1.0, fake, fake, 1.0, fake, 1, 64, 0, 64, 16, 16, 4, 64, 4, fake, fake, 0,
                           None, None) == 1
     assert L.indexer_topk_max_entries(4, 32) == 0
+    # fused decode update: fp32 rows take the separate calls
+    assert L.csa_decode_update(*([fake] * 8), 0, 1, 128, 64, 4, 4, 128, 64, *([fake] * 12), 1.0, fake, None) == 2
     # attention: unsupported head dim
     assert L.sparse_attn_fwd(fake, fake, fake, fake, None, 1.0, 128, 1, 256, 0, 256, 8, 96, 64, 8, 256, fake,
                              fake, None, 1, None, None) == 2
@@ -90,3 +92,18 @@ def test_argument_validation_rejects_before_launch(lib):
     assert L.topk_select(fake, 1, 0, 4, 64, 64, 8, 4, 0, fake, fake, None, 0, None) == 0
     # the wait limit is a host setting (no device access)
     assert L.csa_set_wait_timeout_ns(0) == 0
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every binding's argtypes list has as many entries as the C declaration
+    has parameters (a short list would shift every argument after it)."""
+    from long_context_compressed_compress_b200 import ops
+    txt = open(os.path.join(ROOT, "include", "csa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    decls = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+([a-z_0-9]+)\s*\(([^;]*?)\)\s*;", txt,
+                       flags=re.M | re.S)
+    assert len(decls) >= 15
+    for name, params in decls:
+        params = params.strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        assert len(ops._SIGS[name][0]) == n, (name, n, len(ops._SIGS[name][0]))

@@ -146,3 +146,26 @@ def test_decode_from_empty_cache(L):
     softmax covers only its own block's m logits (no predecessor)."""
     cfg = dataclasses.replace(configs.CSA_DECODE, B=3, T0=0, steps=12)
     run_decode(L, cfg, [0, 1, 2], 12, graph=False)
+
+
+def test_fused_state_update_equals_separate_calls(L):
+    """csa_decode_update (one launch) leaves the carry rings, the window ring,
+    the compressed entries, their NVFP4 keys and q_I's NVFP4 codes exactly as
+    the seven appends, two decode-mode compressions and the quantisation do,
+    over eight steps (two entries emitted), from an empty cache and from a
+    cache of 65536 tokens; the step outputs are identical."""
+    for cfg in (dataclasses.replace(configs.CSA_DECODE, B=3, T0=0, steps=8), SMALL):
+        st = inputs.decode_state(cfg)
+        lays = [L.CsaDecode(cfg, {k: v.cuda() for k, v in st.items()}, cfg.T0, fused_update=f) for f in (True, False)]
+        assert lays[0].fused_update and not lays[1].fused_update
+        assert lays[0].launches < lays[1].launches
+        for step in range(8):
+            x = {k: v.cuda() for k, v in inputs.decode_step_inputs(cfg, step).items()}
+            outs = [lay.step(x).clone() for lay in lays]
+            torch.cuda.synchronize()
+            f, s = lays
+            for n in CARRY:
+                assert torch.equal(f.carry[n], s.carry[n]), n
+            for name in ("ring", "kv_c", "k_fp4", "k_sf", "q_fp4", "q_sf", "idx", "pos"):
+                assert torch.equal(getattr(f, name), getattr(s, name)), (step, name)
+            assert torch.equal(outs[0], outs[1])
