@@ -235,6 +235,22 @@ int indexer_topk(const uint8_t* q_fp4, const uint8_t* q_sf, float q_gscale,
 int indexer_topk_max_entries(int HI, int DI);
 
 /*
+ * csa_validate_indices -- bounds check of an idx tensor before the attention
+ * gathers with it (the layer drivers' check mode; [cf-1] §3.1: a query
+ * attends to top-k entries among those it can see).  Row r of the chunk
+ * (position p = q_pos0[b] + row0 + r) sees n = min(S, (p+1)/m) entries; a
+ * valid row holds entries in [0, n), strictly ascending, then -1 padding.
+ *   idx int32 [B, T_chunk, k]; status: caller device word
+ * A violation writes CSA_ERR_INVALID_ARG | site << 8 to *status (the first
+ * one is kept; site 1: entry outside [-1, n), 2: valid entries out of order,
+ * 3: a valid entry after -1 padding).  The kernel only reads idx; it never
+ * traps.
+ */
+int csa_validate_indices(const int32_t* idx, int B, int T_chunk, int k, int S,
+                         int m, int row0, const int32_t* q_pos0,
+                         int32_t* status, csa_stream_t stream);
+
+/*
  * topk_select_noalloc -- topk_select for callers that cannot allocate device
  * memory (no workspace argument).  The pages have no counterpart to this call;
  * it exists only for allocator-free callers.  Same arguments, layouts, result

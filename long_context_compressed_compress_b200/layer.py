@@ -16,6 +16,8 @@ HCA prefill (§3.2, §3.3):
 """
 from __future__ import annotations
 
+import os
+
 import torch
 
 from . import ops
@@ -35,11 +37,23 @@ def _no_timer(name):
     return _Null()
 
 
+def _check_mode(check):
+    return bool(int(os.environ.get("CSA_CHECK", "0"))) if check is None else bool(check)
+
+
+def raise_on_status(status):
+    """Raise if a check or a bounded wait recorded an error in ``status``."""
+    v = int(status.item())
+    if v != 0:
+        status.zero_()
+        raise ops.CsaError("device check", v & 0xFF)
+
+
 class CsaPrefill:
     """Buffers + call sequence of one CSA prefill layer.  ``chunk`` bounds the
     query rows scored at once (the score buffer is [B, chunk, S])."""
 
-    def __init__(self, cfg, device="cuda", chunk=None, gscale=1.0, fused=None):
+    def __init__(self, cfg, device="cuda", chunk=None, gscale=1.0, fused=None, check=None):
         self.cfg = cfg
         c = cfg
         dt = _DT[c.dtype]
@@ -66,6 +80,10 @@ class CsaPrefill:
         self.lse = None
         self.q_pos0 = torch.zeros((c.B,), dtype=torch.int32, device=device)
         self.launches = 3 + (2 if self.fused else 3) * ((c.T + self.chunk - 1) // self.chunk)
+        # check mode (argument, or CSA_CHECK=1 in the environment): every idx
+        # chunk is bounds-checked before the attention gathers with it
+        self.check = _check_mode(check)
+        self.status = torch.zeros((1,), dtype=torch.int32, device=device) if self.check else None
 
     def run(self, x, keep_idx=None, timer=None):
         """x: dict of device tensors (input generator order).  If ``keep_idx`` is a
@@ -94,11 +112,15 @@ class CsaPrefill:
                                       c.m, row0=r0, T_chunk=tc, q_gscale=self.g, k_gscale=self.g)
                 with t("topk_select"):
                     ops.topk_select(sc, ix, c.S, c.m, self.q_pos0, row0=r0)
+            if self.check:
+                ops.validate_indices(ix, c.S, c.m, self.q_pos0, self.status, row0=r0)
             with t("sparse_attn_fwd"):
                 ops.sparse_attn_fwd(x["q"], self.kv_c, ix, x["kv_raw"], x["sink"], c.tau, c.W, self.q_pos0,
                                     self.out, self.lse, row0=r0, T_chunk=tc)
             if keep_idx is not None:
                 keep_idx[:, r0:r0 + tc].copy_(ix)
+        if self.check:
+            raise_on_status(self.status)
         return self.out
 
 
@@ -154,7 +176,7 @@ class CsaDecode:
     captured once in a CUDA graph (``capture``) and replayed.
     """
 
-    def __init__(self, cfg, state, T0, device="cuda", gscale=1.0, with_lse=False, fused_update=None):
+    def __init__(self, cfg, state, T0, device="cuda", gscale=1.0, with_lse=False, fused_update=None, check=None):
         self.cfg = c = cfg
         dt = _DT[c.dtype]
         self.dt = dt
@@ -200,6 +222,11 @@ class CsaDecode:
         self.fused_update = can_fuse if fused_update is None else bool(fused_update)
         # multi-CTA top-k: workspace memset + three kernels
         self.launches = (1 if self.fused_update else 6 + 2 + 1 + 1) + 1 + (4 if nws else 1) + 1 + 1
+        # check mode: idx is bounds-checked on the device every step; the
+        # caller reads the verdict with raise_on_status(self.status)
+        self.check = _check_mode(check)
+        self.status = torch.zeros((1,), dtype=torch.int32, device=device) if self.check else None
+        self.launches += 1 if self.check else 0
         self.graph = None
         self.x = None
 
@@ -232,6 +259,8 @@ class CsaDecode:
                               self.score, self.cap, c.m, q_gscale=self.g, k_gscale=self.g)
         with t("topk_select"):
             ops.topk_select(self.score, self.idx, self.cap, c.m, self.pos, workspace=self.ws)
+        if self.check:
+            ops.validate_indices(self.idx, self.cap, c.m, self.pos, self.status)
         sink = x["sink"] if "sink" in x else self.sink
         with t("sparse_attn_fwd"):
             ops.sparse_attn_fwd(x["q"].view(-1, 1, c.H, x["q"].shape[-1]), self.kv_c, self.idx, self.ring, sink,

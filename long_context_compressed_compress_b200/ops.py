@@ -50,6 +50,7 @@ _SIGS = {
     "topk_select": ([P, I, I, I, I, I, I, I, I, P, P, P, SZ, P], I),
     "indexer_topk": ([P, P, F, P, P, F, P, I, I, I, I, I, I, I, I, I, P, P, I, P, P], I),
     "indexer_topk_max_entries": ([I, I], I),
+    "csa_validate_indices": ([P, I, I, I, I, I, I, P, P, P], I),
     "topk_workspace_size": ([I, I, I, I], SZ),
     "topk_select_noalloc": ([P, I, I, I, I, I, I, I, I, P, P, P], I),
     "sparse_attn_fwd": ([P, P, P, P, P, F, I, I, I, I, I, I, I, I, I, I, P, P, P, I, P, P], I),
@@ -167,6 +168,14 @@ def indexer_topk(q_fp4, q_sf, k_fp4, k_sf, w, q_pos0, idx, S, m, row0=0, T_chunk
 
 def indexer_topk_max_entries(HI, DI):
     return int(lib.indexer_topk_max_entries(HI, DI))
+
+
+def validate_indices(idx, S, m, q_pos0, status, row0=0, stream=None):
+    """Check idx [B, T_chunk, k] (entries in [0, visible), ascending, then -1);
+    a violation is recorded in the device word ``status`` (int32 [1])."""
+    B, T_chunk, k = idx.shape
+    _check("csa_validate_indices", lib.csa_validate_indices(_ptr(idx), B, T_chunk, k, S, m, row0, _ptr(q_pos0),
+                                                            _ptr(status), _stream(stream)))
 
 
 def topk_select_noalloc(score, idx, S, m, q_pos0, row0=0, stream=None):
