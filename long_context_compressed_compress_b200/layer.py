@@ -84,6 +84,7 @@ class CsaPrefill:
         # chunk is bounds-checked before the attention gathers with it
         self.check = _check_mode(check)
         self.status = torch.zeros((1,), dtype=torch.int32, device=device) if self.check else None
+        self.launches += ((c.T + self.chunk - 1) // self.chunk) if self.check else 0
 
     def run(self, x, keep_idx=None, timer=None):
         """x: dict of device tensors (input generator order).  If ``keep_idx`` is a
