@@ -2,10 +2,10 @@
 
 Sizes span several tiles plus ragged tails.  Tolerances:
   * NVFP4 codes/scales and top-k indices: bit-exact;
-  * fp32 results: 1e-5 * max(1, |ref|) (north-star fp32 bound);
+  * fp32 results: 1e-5 * max(1, |ref|) (the fp32 acceptance bound);
   * bf16 results: the bf16 rounding of the oracle value within one bf16 ulp
     for single-rounding steps (compressors, scores), 2e-2 max-abs for
-    attention outputs (spec bf16 bound).
+    attention outputs (the bf16 acceptance bound).
 """
 import numpy as np
 import pytest

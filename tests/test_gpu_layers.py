@@ -1,7 +1,7 @@
 """End-to-end parity of whole layers (GPU path through the C ABI vs the CPU
 oracle) on the workload recipes, plus determinism and batch invariance.
 
-Acceptance (north-star):
+Acceptance:
   * index sets: mean over rows of |I_gpu & I_orc| / |I_orc| >= 99.5%, and every
     disagreement is a near-tie: the oracle scores of the swapped entries lie
     within 2 bf16 ulps (bf16 scores) or 1e-6 relative (fp32 scores) of the

@@ -24,7 +24,7 @@ def _rand(*shape):
 
 def test_csa_one_hot_gate_selects_single_token_current_block():
     """With one gate logit far above the rest, the entry equals that token's row:
-    the ``a`` row when the token is in the current block (spec invariant)."""
+    the ``a`` row when the token is in the current block (an invariant of the definition)."""
     T, D, m = 32, 8, 4
     a, b = _rand(T, D), _rand(T, D)
     for i in range(T // m):
@@ -303,7 +303,7 @@ def _sdpa(q, k, v, scale, mask=None, causal=False):
 
 
 def test_hca_ratio_one_no_window_no_sink_equals_causal_sdpa():
-    """Spec invariant: HCA with ratio 1 is causal dense attention."""
+    """Invariant: HCA with ratio 1 is causal dense attention."""
     B, T, H, D, tau = 2, 37, 3, 8, 0.3
     q, x = _rand(B, T, H, D), _rand(B, T, D)
     e = oracle.hca_compress(x, _rand(B, T, D), 1)          # ratio 1: e == x
@@ -328,7 +328,7 @@ def test_window_only_equals_banded_sdpa():
 
 
 def test_csa_with_k_covering_all_entries_equals_dense():
-    """Spec invariant: with k >= S, CSA equals dense attention over entries."""
+    """Invariant: with k >= S, CSA equals dense attention over entries."""
     B, T, H, D, m, W = 1, 64, 4, 8, 4, 7
     S = T // m
     q, kv_c, raw = _rand(B, T, H, D), _rand(B, S, D), _rand(B, T, D)
@@ -343,7 +343,7 @@ def test_csa_with_k_covering_all_entries_equals_dense():
 
 
 def test_sink_closed_form_only_lowers_mass():
-    """out_sigma = out_nosink * Z / (Z + e^sigma), Z = e^lse (spec: the sink
+    """out_sigma = out_nosink * Z / (Z + e^sigma), Z = e^lse (the sink
     only lowers attention mass)."""
     B, T, H, D, m, W = 1, 48, 5, 8, 4, 16
     S = T // m
