@@ -48,3 +48,22 @@ def test_workloads_use_the_printed_values():
     assert configs.CSA_PREFILL_K1024.k == int(v["csa_top_k"])
     # bf16 scores in the bf16 workloads (the fp32 workload keeps fp32 scores)
     assert v["index_score_dtype"] == "bf16" and configs.CSA_PREFILL.dtype == "bf16"
+
+
+def test_bench_algorithmic_work_closed_forms():
+    """The bench's per-launch algorithmic work equals closed forms: visible
+    (row, entry) pairs sum min(S, (t+1) // m) over rows; attended rows add
+    min(k, visible) + min(W, t + 1); attention FLOPs are 4 D H per attended row."""
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    c = configs.scaled(configs.CSA_PREFILL, T=1000)
+    w = bench.algorithmic_work(c)
+    vis = [min(c.S, (t + 1) // c.m) for t in range(c.T)]
+    rows = sum(min(c.k, v) + min(c.W, t + 1) for t, v in enumerate(vis))
+    assert w["indexer_pairs"] == c.B * sum(vis)
+    assert w["attn_rows"] == c.B * rows
+    assert w["attn_flops"] == c.B * 4.0 * c.H * c.D * rows
+    assert w["topk_bytes"] == c.B * (sum(vis) * 2 + c.T * c.k * 4)
+    assert w["indexer_topk_bytes"] == c.B * (c.T * c.HI * (c.DI // 2 + c.DI // 16 + 4) +
+                                             c.S * (c.DI // 2 + c.DI // 16) + c.T * c.k * 4)
